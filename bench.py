@@ -1,0 +1,403 @@
+"""Benchmark: effective TFLOP/s of block-sparse varlen attention, forward +
+backward, on one of the five workloads (default C3: BNSD B=2, N1=N2=32,
+S=8192, D=128, bf16, block (128,512), fully dense index -- the tensor-core
+roofline workload).
+
+A step is one forward (bsa_fwd: index compaction, work list, attention)
+followed by one backward (bsa_bwd: inverse index, work list, preprocess,
+KV-major dK/dV with dQ reduction, dQ conversion) on inputs resident in HBM,
+the backward consuming the forward's out and lse.  Effective FLOPs count
+kept (q head, valid q token, valid kv token) pairs only: 4*D per pair
+forward, 10*D backward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C3] [--impl ours|reference]
+
+Under torchrun each rank runs an independent replica of the workload on its
+own GPU (the path shards by batch / kv-head group with no exchange), so the
+job value is N x the per-replica work over the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "effective TFLOP/s (selected blocks only) fwd and bwd; % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+DESCR = {
+    1: "C1: BNSD B=1 N1=N2=2 S=512 D=64 bf16, block (128,128), random index [1,2,4,4]",
+    2: "C2: TND B=4 lens U[256,3072] N1=16 N2=4 D=128 bf16, block (128,128), 25% + diagonal",
+    3: "C3: BNSD B=2 N1=N2=32 S=8192 D=128 bf16, block (128,512), dense index [2,32,64,16]",
+    4: "C4: BNSD B=1 N1=N2=24 S=32768 D=128 bf16, block (128,128), sink+diag+14 random of 256",
+    5: "C5: TND q B=8 lens U[512,4096] + paged KV [P,128,8,128] fp16, N1=32 N2=8, top-8 blocks",
+}
+# kernels this library launches per step (forward 5, backward 12)
+LAUNCHES_PER_STEP = 17
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            d = json.load(f)
+        return d, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def _pairs(p):
+    from workloads.gen import NO_BLOCK  # noqa: F401  (structure only)
+    # kept pairs = sum over (head, query block row) of valid q rows x valid
+    # kv tokens of the accepted blocks; the index of every workload here is
+    # valid (ascending, in range), so accepted = present entries
+    idx = p.index.view(torch.int16).numpy().view(np.uint16).astype(np.int64)
+    g = p.N1 // p.N2
+    total = 0
+    lens_q, lens_kv = p.lens_q, p.lens_kv
+    if p.layout_q == "BNSD":
+        for b in range(p.B):
+            for hi in range(p.Hidx):
+                heads = 1 if p.Hidx == p.N1 else g
+                for i in range(idx.shape[2]):
+                    rows = min(p.BQ, lens_q[b] - i * p.BQ)
+                    e = idx[b, hi, i]
+                    e = e[e != 0xFFFF]
+                    cols = int(np.minimum(p.BKV, lens_kv[b] - e * p.BKV).sum())
+                    total += heads * rows * cols
+    else:
+        off = 0
+        for b in range(p.B):
+            nq = -(-lens_q[b] // p.BQ)
+            for hi in range(p.Hidx):
+                heads = 1 if p.Hidx == p.N1 else g
+                for i in range(nq):
+                    rows = min(p.BQ, lens_q[b] - i * p.BQ)
+                    e = idx[hi, off + i]
+                    e = e[e != 0xFFFF]
+                    cols = int(np.minimum(p.BKV, lens_kv[b] - e * p.BKV).sum())
+                    total += heads * rows * cols
+            off += nq
+    return total
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.25)
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for l in getattr(self, "lines", []):
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- oracle leg
+def _oracle_subproblem(cfg: int, q_rows: int):
+    """A bounded slice of the workload for the CPU oracle: batch 0, head 0,
+    the first q_rows query rows against the full key range."""
+    import workloads
+    from workloads.gen import make_problem, pat_dense
+    p = workloads.make_config(cfg)
+    if p.layout_q != "BNSD":
+        raise SystemExit("CPU baseline slice is defined for the BNSD workloads")
+    S = p.q.shape[2]
+    q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
+    sub = make_problem(B=1, N1=1, N2=1, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
+                       BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale)
+    sub.q = p.q[:1, :1, :q_rows].contiguous()
+    sub.k = p.k[:1, :1].contiguous()
+    sub.v = p.v[:1, :1].contiguous()
+    sub.dout = p.dout[:1, :1, :q_rows].contiguous()
+    sub.index = p.index[:1, :1, :q_rows // p.BQ].contiguous()
+    sub.lens_q = [q_rows]
+    return sub
+
+
+def _oracle_step(sub):
+    import oracle
+    o = oracle.Oracle(sub)
+    t = time.perf_counter()
+    out, lse, _ = o.fwd()
+    o.bwd(out, sub.dout, lse)
+    return time.perf_counter() - t
+
+
+def _oracle_rate(cfg: int, target_s: float):
+    """Calibrate the slice to ~target_s per step; returns (sub, pairs, seconds)."""
+    sub = _oracle_subproblem(cfg, 128)
+    t = _oracle_step(sub)
+    rows = int(128 * max(1.0, target_s / max(t, 1e-3)))
+    sub = _oracle_subproblem(cfg, rows)
+    return sub, _pairs(sub)
+
+
+def cpu_baseline(cfg: int, target_s: float = 12.0):
+    sub, pairs = _oracle_rate(cfg, target_s)
+    t = _oracle_step(sub)
+    flops = 14 * sub.D * pairs
+    return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _omp_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle fwd+bwd on batch 0, head 0, first {sub.q.shape[2]} query rows "
+                      f"x {sub.k.shape[2]} keys of {DESCR[cfg].split(':')[0]} ({pairs} kept pairs, "
+                      f"{t:.1f} s)"}
+
+
+def _omp_threads():
+    n = os.environ.get("OMP_NUM_THREADS")
+    return int(n) if n and n.isdigit() else (os.cpu_count() or 1)
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    sub, pairs = _oracle_rate(args.config, 2.0)
+    for _ in range(args.warmup):
+        _oracle_step(sub)
+    ts = [_oracle_step(sub) for _ in range(args.steps)]
+    total = sum(ts)
+    flops = 14 * sub.D * pairs
+    val = flops * args.steps / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": DESCR[args.config], "sample": "see cpu_baseline"},
+            "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _omp_threads(),
+                             "kind": "oracle",
+                             "sample": f"batch 0, head 0, first {sub.q.shape[2]} query rows "
+                                       f"({pairs} kept pairs) per step"},
+            "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# -------------------------------------------------------------------- GPU leg
+def run_ours(args):
+    import block_sparse_variable_b200 as bsa
+    import workloads
+    from tests.harness import params_of
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    p = workloads.make_config(args.config)
+    pairs = _pairs(p)
+    P = params_of(p)
+    to = lambda t: None if t is None else t.to(dev)  # noqa: E731
+    q, k, v, dout, index = (to(getattr(p, n)) for n in ("q", "k", "v", "dout", "index"))
+    opt = dict(cu_seqlens_q=to(p.cu_q), cu_seqlens_kv=to(p.cu_kv), seqused_kv=to(p.seqused_kv),
+               block_table=to(p.block_table))
+    out = torch.empty_like(q)
+    lse = torch.empty((q.shape[0], q.shape[1], q.shape[2]) if p.layout_q == "BNSD"
+                      else (q.shape[0], q.shape[1]), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    wsf = torch.empty(bsa.bsa_fwd_get_workspace(q, k, v, index, P, out=out, lse=lse, **opt),
+                      dtype=torch.uint8, device=dev)
+    wsb = torch.empty(bsa.bsa_bwd_get_workspace(q, k, v, out, dout, lse, index, P, dq=dq, dk=dk,
+                                                dv=dv, **opt), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bsa.bsa_fwd(q, k, v, index, P, out=out, lse=lse, workspace=wsf, stream=stream, **opt)
+        bsa.bsa_bwd(q, k, v, out, dout, lse, index, P, dq=dq, dk=dk, dv=dv, workspace=wsb,
+                    stream=stream, **opt)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    flags = bsa.bsa_read_status(wsf) | bsa.bsa_read_status(wsb)
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index if world == 1 else local) as clk:
+        start.record(stream)
+        for s in range(args.steps):
+            ev[s][0].record(stream)
+            bsa.bsa_fwd(q, k, v, index, P, out=out, lse=lse, workspace=wsf, stream=stream, **opt)
+            ev[s][1].record(stream)
+            bsa.bsa_bwd(q, k, v, out, dout, lse, index, P, dq=dq, dk=dk, dv=dv, workspace=wsb,
+                        stream=stream, **opt)
+            ev[s][2].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    ms = start.elapsed_time(stop)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    if dist:
+        t = torch.tensor([ms, fwd_ms, bwd_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, fwd_ms, bwd_ms = (float(x) for x in t.tolist())
+
+    # ---- end to end through the C ABI from pinned host buffers
+    hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
+    hidx = index.cpu().pin_memory()
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h_dq = torch.empty(dq.shape, dtype=dq.dtype).pin_memory()
+    h_dk = torch.empty(dk.shape, dtype=dk.dtype).pin_memory()
+    h_dv = torch.empty(dv.shape, dtype=dv.dtype).pin_memory()
+    e2e_steps = max(2, min(args.steps, 5))
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo, hidx))
+    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse, h_dq, h_dk, h_dv))
+
+    def e2e_step():
+        for d_, h_ in ((q, hq), (k, hk), (v, hv), (dout, hdo), (index, hidx)):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in ((h_out, out), (h_lse, lse), (h_dq, dq), (h_dk, dk), (h_dv, dv)):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank == 0:
+        peaks, which = _peaks()
+        D = p.D
+        step_flops = 14 * D * pairs
+        ms_step = ms / args.steps
+        value = world * step_flops / (ms_step * 1e-3) / 1e12
+        fwd_tf = 4 * D * pairs / (fwd_ms * 1e-3) / 1e12
+        bwd_tf = 10 * D * pairs / (bwd_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
+        achieved = bwd_tf if dominant == "bwd" else fwd_tf
+        traffic = _traffic_from_profiles(args.config, dominant)
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if p.dtype == torch.bfloat16 else "f16", "data": "synthetic",
+            "config": {"workload": DESCR[args.config], "kept_pairs_per_replica": pairs,
+                       "parallelism": f"replicas x{world} (no exchange)",
+                       "l2": "inputs larger than L2 (q/k/v/dout %d MiB each)"
+                             % (q.numel() * q.element_size() >> 20)},
+            "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
+            "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+            "pct_of_peak": round(100 * value / world / peak, 2),
+            "roofline": {"bound": "tensor", "kernel": f"bsa_{dominant} call (main kernel + prep)",
+                         "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                         "frac": round(achieved / peak, 4), "peak_source": f"{which} bf16 burst",
+                         "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
+                         "traffic": traffic},
+            "e2e": {"value": round(world * step_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": round(e2e_ms, 3)},
+            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "status_flags": flags,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args.config)
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _traffic_from_profiles(cfg, which):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d.get(f"C{cfg}", {}).get(which)
+    except (OSError, ValueError):
+        return None
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=lambda s: int(s.lstrip("Cc")), default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,349 @@
+// prep.cu -- on-device builders that run before the attention kernels:
+//   * batch geometry from cu_seqlens / seqused_kv (lengths, block counts,
+//     packed-row offsets, row -> batch maps);
+//   * index compaction: drop 0xFFFF and invalid entries of every index row
+//     (BlitzSparseAttention "sabi": ascending ids, 0xFFFF = unused slot) and
+//     count the forward work of each (head, 128-row query slice);
+//   * the KV-major inverse of the index (GenericBlockSparseAttention,
+//     layoutSparsePattern 5/7: the query blocks that chose each kv block),
+//     as CSR, plus the backward work of each (kv head, 128-row kv slice);
+//   * the load-balanced work lists: item ids sorted by cost descending then
+//     id ascending (longest first, ties head-major), by a per-CTA bitonic
+//     sort of 4096-key chunks followed by a merge by rank.
+#include <cuda_runtime.h>
+
+#include "bsa_internal.h"
+
+namespace bsa {
+namespace {
+
+__device__ __forceinline__ int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+__global__ void k_geometry(Problem p) {
+  __shared__ uint32_t sflags;
+  uint32_t *st = p.status;
+  for (int i = threadIdx.x; i < kStWords; i += blockDim.x) st[i] = 0;
+  for (int64_t r = threadIdx.x; r < p.Rg; r += blockDim.x) p.row_batch[r] = -1;
+  for (int64_t r = threadIdx.x; r < p.tk_max; r += blockDim.x) p.kb_batch[r] = -1;
+  if (threadIdx.x == 0) sflags = 0;
+  __syncthreads();
+
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    uint32_t f = 0;
+    int64_t qlen = p.Sq, q0 = 0, kvst = 0, kv0 = 0;
+    if (p.q_layout == BSA_LAYOUT_TND) {
+      const int64_t a = p.cu_q[b], e = p.cu_q[b + 1];
+      if (a < 0 || e < a || e > p.Tq) { f |= BSA_FLAG_BAD_SEQLEN; qlen = 0; }
+      else { qlen = e - a; q0 = a; }
+    }
+    if (p.kv_layout == BSA_LAYOUT_BNSD) {
+      kvst = p.Skv;
+    } else if (p.kv_layout == BSA_LAYOUT_PA_BBND) {
+      kvst = int64_t(p.max_pages) * p.page_size;
+    } else {
+      const int64_t a = p.cu_kv[b], e = p.cu_kv[b + 1];
+      if (a < 0 || e < a || e > p.Tkv) { f |= BSA_FLAG_BAD_SEQLEN; kvst = 0; }
+      else { kvst = e - a; kv0 = a; }
+    }
+    int64_t kvlen = kvst;
+    if (p.seqused_kv) {
+      const int64_t u = p.seqused_kv[b];
+      if (u < 0 || u > kvst) { f |= BSA_FLAG_BAD_SEQLEN; kvlen = 0; }
+      else kvlen = u;
+    }
+    BatchInfo bi;
+    bi.qlen = int32_t(qlen);
+    bi.kvlen = int32_t(kvlen);
+    bi.nq = int32_t(cdiv64(qlen, p.BQ));
+    bi.nk = int32_t(cdiv64(kvlen, p.BKV));
+    bi.qoff = 0;
+    bi.koff = 0;
+    bi.q_tok0 = q0;
+    bi.kv_tok0 = kv0;
+    // rows of dk/dv the backward may write: the stored rows, or under paging
+    // the rows of the pages that cover the used length
+    bi.kvst = p.kv_layout == BSA_LAYOUT_PA_BBND
+                  ? int32_t(cdiv64(kvlen, p.page_size) * p.page_size)
+                  : int32_t(kvst);
+    bi.pad = 0;
+    p.batch[b] = bi;
+    if (f) atomicOr(&sflags, f);
+  }
+  __syncthreads();
+
+  if (threadIdx.x == 0) {
+    int64_t qo = 0, ko = 0;
+    uint32_t f = 0;
+    for (int b = 0; b < p.B; ++b) {
+      BatchInfo &bi = p.batch[b];
+      if (p.q_layout == BSA_LAYOUT_TND) { bi.qoff = int32_t(qo); qo += bi.nq; }
+      else { bi.qoff = b * p.R; qo += bi.nq; }
+      if (ko + bi.nk > p.tk_max) {  // only inconsistent cu_seqlens_kv reach this
+        f |= BSA_FLAG_BAD_SEQLEN;
+        bi.nk = 0;
+        bi.kvlen = 0;
+      }
+      bi.koff = int32_t(ko);
+      ko += bi.nk;
+    }
+    if (p.q_layout == BSA_LAYOUT_TND && qo > p.R) f |= BSA_FLAG_BAD_INDEX;
+    st[kStTK] = uint32_t(ko);
+    st[kStSumNq] = uint32_t(qo);
+    if (f) atomicOr(&sflags, f);
+  }
+  __syncthreads();
+
+  for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
+    const BatchInfo bi = p.batch[b];
+    for (int i = 0; i < bi.nq; ++i) {
+      const int64_t r = int64_t(bi.qoff) + i;
+      if (r < p.Rg) p.row_batch[r] = b;
+    }
+    for (int j = 0; j < bi.nk; ++j) p.kb_batch[bi.koff + j] = b;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) st[kStFlags] = sflags;
+}
+
+__device__ __forceinline__ uint64_t make_key(int32_t cost, int64_t id) {
+  return (uint64_t(0xFFFFFFFFu - uint32_t(cost)) << 32) | uint64_t(uint32_t(id));
+}
+
+// one thread per (index head, global q-block row)
+__global__ void k_compact(Problem p, int fwd_keys) {
+  const int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (r >= int64_t(p.Hidx) * p.Rg) return;
+  const int hi = int(r / p.Rg);
+  const int gq = int(r % p.Rg);
+  uint16_t *dst = p.comp + r * p.W;
+  const int b = p.row_batch[gq];
+  int n = 0, cost = 0, i = 0, qlen = 0;
+  if (b >= 0) {
+    const BatchInfo bi = p.batch[b];
+    i = gq - bi.qoff;
+    qlen = bi.qlen;
+    const uint16_t *row = p.q_layout == BSA_LAYOUT_BNSD
+                              ? p.index + b * p.ix_s0 + hi * p.ix_s1 + i * p.ix_s2
+                              : p.index + hi * p.ix_s0 + int64_t(gq) * p.ix_s1;
+    int last = -1;
+    bool bad = false;
+    for (int w = 0; w < p.W; ++w) {
+      const int e = row[w];
+      if (e == kNoBlock) continue;
+      if (e >= bi.nk || e <= last) { bad = true; continue; }
+      dst[n++] = uint16_t(e);
+      last = e;
+      const int rem = bi.kvlen - e * p.BKV;  // > 0 because e < nk
+      cost += min(p.ksl, (rem + kSlice - 1) / kSlice);
+    }
+    if (bad) atomicOr(p.status + kStFlags, BSA_FLAG_BAD_INDEX);
+  }
+  for (int w = n; w < p.W; ++w) dst[w] = kNoBlock;
+  p.ncomp[r] = n;
+  if (!fwd_keys) return;
+  const int h_lo = p.Hidx == p.N1 ? hi : hi * p.g;
+  const int h_hi = p.Hidx == p.N1 ? hi + 1 : h_lo + p.g;
+  int made = 0;
+  for (int h1 = h_lo; h1 < h_hi; ++h1)
+    for (int qs = 0; qs < p.nsub; ++qs) {
+      const int64_t slot = (int64_t(h1) * p.Rg + gq) * p.nsub + qs;
+      const bool exists = b >= 0 && i * p.BQ + qs * kSlice < qlen;
+      p.keys[slot] = exists ? make_key(cost, slot) : kAbsentKey;
+      made += exists;
+    }
+  if (made) atomicAdd(p.status + kStFwdItems, uint32_t(made));
+}
+
+__device__ __forceinline__ bool row_has(const uint16_t *row, int n, int j) {
+  int lo = 0, hi = n;  // ascending row: binary search
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (int(row[mid]) < j) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo < n && int(row[lo]) == j;
+}
+
+// one thread per (index head, kv block); mode 0 counts, mode 1 fills
+__global__ void k_inverse(Problem p, int mode) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= int64_t(p.Hidx) * p.tk_max) return;
+  const int hi = int(idx / p.tk_max);
+  const int gk = int(idx % p.tk_max);
+  const int TK = int(p.status[kStTK]);
+  if (gk >= TK) return;
+  const int b = p.kb_batch[gk];
+  const int64_t li = int64_t(hi) * TK + gk;
+  int cnt = 0, sub = 0;
+  int pos = mode ? p.inv_off[li] : 0;
+  if (b >= 0) {
+    const BatchInfo bi = p.batch[b];
+    const int j = gk - bi.koff;
+    for (int i = 0; i < bi.nq; ++i) {
+      const int64_t gq = int64_t(bi.qoff) + i;
+      if (gq >= p.Rg) break;
+      const int64_t rr = int64_t(hi) * p.Rg + gq;
+      if (row_has(p.comp + rr * p.W, p.ncomp[rr], j)) {
+        if (mode) p.inv_list[pos++] = i;
+        ++cnt;
+        sub += min(p.nsub, (bi.qlen - i * p.BQ + kSlice - 1) / kSlice);
+      }
+    }
+  }
+  if (!mode) {
+    p.inv_cnt[li] = cnt;
+    p.inv_sub[li] = sub;
+  }
+}
+
+// single CTA exclusive scan of inv_cnt[0 .. Hidx*TK) into inv_off
+__global__ void k_scan_offsets(Problem p) {
+  __shared__ int32_t warp_sums[32];
+  __shared__ int32_t carry;
+  const int64_t n = int64_t(p.Hidx) * p.status[kStTK];
+  if (threadIdx.x == 0) carry = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int64_t base = 0; base < n; base += blockDim.x) {
+    const int64_t i = base + threadIdx.x;
+    const int32_t x = i < n ? p.inv_cnt[i] : 0;
+    int32_t s = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane == 31) warp_sums[wid] = s;
+    __syncthreads();
+    if (wid == 0) {
+      int32_t w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int32_t y = __shfl_up_sync(0xffffffffu, w, o);
+        if (lane >= o) w += y;
+      }
+      if (lane < nw) warp_sums[lane] = w;
+    }
+    __syncthreads();
+    const int32_t before = carry + (wid ? warp_sums[wid - 1] : 0) + s - x;
+    if (i < n) p.inv_off[i] = before;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) carry = before + x;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    p.inv_off[n] = carry;
+    p.status[kStNnz] = uint32_t(carry);
+  }
+}
+
+// one thread per backward slot (h2, gk, kv slice)
+__global__ void k_bwd_keys(Problem p) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= p.bwd_slots) return;
+  const int TK = int(p.status[kStTK]);
+  const int64_t live = int64_t(p.N2) * TK * p.ksl;
+  if (idx >= live) { p.keys[idx] = kAbsentKey; return; }
+  const int ks = int(idx % p.ksl);
+  const int gk = int((idx / p.ksl) % TK);
+  const int h2 = int(idx / (int64_t(p.ksl) * TK));
+  const int b = p.kb_batch[gk];
+  bool exists = false;
+  int cost = 0;
+  if (b >= 0) {
+    const BatchInfo bi = p.batch[b];
+    const int j = gk - bi.koff;
+    exists = j * p.BKV + ks * kSlice < bi.kvlen;
+    if (p.Hidx == p.N1) {
+      for (int h1 = h2 * p.g; h1 < (h2 + 1) * p.g; ++h1) cost += p.inv_sub[int64_t(h1) * TK + gk];
+    } else {
+      cost = p.g * p.inv_sub[int64_t(h2) * TK + gk];
+    }
+  }
+  p.keys[idx] = exists ? make_key(cost, idx) : kAbsentKey;
+  if (exists) atomicAdd(p.status + kStBwdItems, 1u);
+}
+
+// bitonic sort of one kSortChunk-key chunk in shared memory (ascending)
+__global__ void __launch_bounds__(1024) k_sort_chunks(const uint64_t *keys, uint64_t *sorted,
+                                                      int64_t slots) {
+  __shared__ uint64_t s[kSortChunk];
+  const int64_t base = int64_t(blockIdx.x) * kSortChunk;
+  for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x)
+    s[i] = base + i < slots ? keys[base + i] : kAbsentKey;
+  __syncthreads();
+  for (int k = 2; k <= kSortChunk; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint64_t a = s[i], c = s[ixj];
+          const bool up = (i & k) == 0;
+          if ((a > c) == up) { s[i] = c; s[ixj] = a; }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x) sorted[base + i] = s[i];
+}
+
+// final position of every real key = its place in its chunk + the keys
+// below it in every other chunk (keys are unique: the id is in the low word)
+__global__ void k_rank(const uint64_t *sorted, int64_t nchunks, int32_t *items) {
+  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= nchunks * kSortChunk) return;
+  const uint64_t key = sorted[idx];
+  if (key == kAbsentKey) return;
+  const int64_t c = idx / kSortChunk;
+  int64_t rank = idx - c * kSortChunk;
+  for (int64_t o = 0; o < nchunks; ++o) {
+    if (o == c) continue;
+    const uint64_t *a = sorted + o * kSortChunk;
+    int lo = 0, hi = kSortChunk;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (a[mid] < key) lo = mid + 1;
+      else hi = mid;
+    }
+    rank += lo;
+  }
+  items[rank] = int32_t(uint32_t(key & 0xFFFFFFFFu));
+}
+
+}  // namespace
+
+cudaError_t launch_prep_geometry(const Problem &p, cudaStream_t s) {
+  k_geometry<<<1, 1024, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_compact(const Problem &p, bool fwd_keys, cudaStream_t s) {
+  const int64_t n = int64_t(p.Hidx) * p.Rg;
+  if (n > 0) {
+    k_compact<<<unsigned((n + 255) / 256), 256, 0, s>>>(p, fwd_keys ? 1 : 0);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sort_items(const Problem &p, int64_t slots_pad, int32_t *items, cudaStream_t s) {
+  const bool fwd = items == p.fwd_items;
+  const int64_t slots = fwd ? p.fwd_slots : p.bwd_slots;
+  const int64_t nchunks = slots_pad / kSortChunk;
+  if (nchunks == 0) return cudaGetLastError();
+  k_sort_chunks<<<unsigned(nchunks), 1024, 0, s>>>(p.keys, p.sorted, slots);
+  k_rank<<<unsigned((nchunks * kSortChunk + 255) / 256), 256, 0, s>>>(p.sorted, nchunks, items);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_prep_inverse(const Problem &p, cudaStream_t s) {
+  const int64_t n = int64_t(p.Hidx) * p.tk_max;
+  const unsigned grid = unsigned((n + 255) / 256);
+  if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 0);
+  k_scan_offsets<<<1, 1024, 0, s>>>(p);
+  if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 1);
+  if (p.bwd_slots > 0) k_bwd_keys<<<unsigned((p.bwd_slots + 255) / 256), 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

@@ -1,0 +1,233 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block-sparse variable-length
+ * FlashAttention library (libbsa.so).
+ *
+ * The operation (BlockSparseAttentionGrad README, "Formula"; GenericBlock-
+ * SparseAttention article, "sparse attention mechanism"):
+ *
+ *     out = softmax(scale * Q * K_sparse^T) * V_sparse
+ *
+ * where query block i (BQ rows) attends only to the KV blocks (BKV rows)
+ * listed in its row of a uint16 block index (BlitzSparseAttention article,
+ * "sabi" section: ascending batch-local KV block ids, unused slots 0xFFFF).
+ * The forward pass also returns the per-row natural-log log-sum-exp of the
+ * scaled scores (same article, "softmax_lse output"; its all-ones example
+ * fixes lse = ln S + sqrt(D) for S keys and D = head dim at scale 1/sqrt(D)).
+ * The backward pass (BlockSparseAttentionGrad README, "Formula") recomputes
+ * P from the LSE and returns dQ, dK, dV:
+ *     softmax_grad = rowsum(dOut o out), dP = dOut V^T,
+ *     dS = P o (dP - softmax_grad), dV = P^T dOut,
+ *     dQ = dS K scale, dK = dS^T Q scale.
+ *
+ * API shape: two calls per pass, as in the aclnn two-phase interface
+ * (aclnnFlashAttentionUnpaddingScoreGradV2 article, sections 3 and 5): a
+ * *_get_workspace call validates every descriptor and returns the scratch
+ * size, then the exec call runs on a CUDA stream.  There is no executor
+ * object: the library is stateless and every argument is passed again.
+ *
+ * Ownership: the caller owns every buffer, including the workspace (device
+ * memory, at least the returned size, 256-byte aligned).  The library
+ * allocates nothing and keeps no state between calls.  One workspace must
+ * not be used by two calls that may overlap on the GPU.
+ *
+ * Errors: every entry point returns a bsa_status and never aborts.  Host
+ * validation covers shapes, strides, dtypes, layouts and attributes; the
+ * *values* of cu_seqlens, seqused_kv, the index and the block table are not
+ * read on the host (GenericBlockSparseAttention article, "values are not
+ * checked at tiling").  The device skips invalid values and records them as
+ * BSA_FLAG_* bits in the workspace status word, read with bsa_read_status.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------- tensors */
+enum {
+  BSA_F16 = 1,
+  BSA_BF16 = 2,
+  BSA_F32 = 3,
+  BSA_U16 = 4,
+  BSA_I32 = 5,
+  BSA_I64 = 6
+};
+
+/* A strided view of device memory.  data == NULL (or a NULL descriptor
+ * pointer) means "absent" for optional arguments.  Strides are in elements;
+ * the last dimension must be contiguous (stride 1). */
+typedef struct bsa_tensor {
+  void *data;
+  int32_t dtype;
+  int32_t ndim;
+  int64_t shape[4];
+  int64_t stride[4];
+} bsa_tensor;
+
+/* Layouts (BlockSparseAttentionGrad README, "layouts"; GenericBlockSparse-
+ * Attention article, "Paged Attention"):
+ *   BNSD     q [B, N1, Sq, D],  kv [B, N2, Skv, D]
+ *   TND      q [Tq, N1, D],     kv [Tkv, N2, D]; batch b is rows
+ *            cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *   PA_BBND  kv only: [num_pages, page_size, N2, D]; kv token u of batch b
+ *            is page block_table[b][u / page_size], row u % page_size. */
+enum { BSA_LAYOUT_BNSD = 0, BSA_LAYOUT_TND = 1, BSA_LAYOUT_PA_BBND = 2 };
+
+typedef struct bsa_params {
+  int32_t q_layout;       /* BSA_LAYOUT_BNSD or BSA_LAYOUT_TND */
+  int32_t kv_layout;      /* BNSD (needs q BNSD), TND, or PA_BBND (needs q TND) */
+  int64_t num_heads;      /* N1 */
+  int64_t num_kv_heads;   /* N2; 0 means N1.  N1 % N2 == 0 (GQA) */
+  int64_t block_shape[2]; /* {BQ, BKV}, each in {128, 256, 512, 1024} */
+  double scale;           /* 0 means 1/sqrt(D) */
+  int32_t return_lse;     /* forward only: write lse when non-zero */
+} bsa_params;
+
+/* Status codes: the first three echo the aclnn codes the pages list
+ * (161001 null pointer, 161002 invalid parameter, 561103 inner error). */
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_NULLPTR = 161001,       /* a required pointer or descriptor is NULL */
+  BSA_ERR_PARAM_INVALID = 161002, /* shapes / strides / dtypes / attributes disagree */
+  BSA_ERR_UNSUPPORTED = 161003,   /* valid request outside what this build supports */
+  BSA_ERR_WORKSPACE = 161004,     /* workspace NULL, misaligned or too small */
+  BSA_ERR_CUDA = 561000,          /* a kernel launch or CUDA call failed */
+  BSA_ERR_INNER = 561103          /* internal inconsistency */
+} bsa_status;
+
+/* Bits of the device status word (bsa_read_status). */
+#define BSA_FLAG_BAD_INDEX 0x1u   /* an index entry >= ceil(kvlen/BKV), not ascending,
+                                     or more query blocks than index rows (TND) */
+#define BSA_FLAG_BAD_SEQLEN 0x2u  /* cu_seqlens / seqused_kv contradict the storage */
+#define BSA_FLAG_BAD_PAGE 0x4u    /* a block-table entry outside [0, num_pages) */
+#define BSA_FLAG_TIMEOUT 0x8u     /* a bounded device wait gave up (pipeline fault) */
+
+/* ------------------------------------------------------------- forward */
+/* Arguments:
+ *   q       BNSD [B,N1,Sq,D] or TND [Tq,N1,D], F16 or BF16, D in {64, 128}
+ *   k, v    BNSD [B,N2,Skv,D], TND [Tkv,N2,D] or PA_BBND [P,page,N2,D];
+ *           same dtype as q; page % 128 == 0
+ *   index   U16. BNSD q: [B, Hidx, ceil(Sq/BQ), W]; TND q: [Hidx, R, W] with
+ *           the rows of batch b after the ceil(qlen/BQ) rows of every earlier
+ *           batch.  Hidx == N1 (own row per q head) or N2 (the group of q
+ *           heads sharing a kv head shares the row).  Entries are batch-local
+ *           kv block ids; 0xFFFF = unused slot.
+ *   cu_seqlens_q   I64 [B+1], required for TND q (prefix sums, [0] == 0)
+ *   cu_seqlens_kv  I64 [B+1], required for TND kv, absent otherwise
+ *   seqused_kv     I32 [B], optional; required for PA_BBND.  kv tokens at or
+ *                  past seqused_kv[b] are ignored.
+ *   block_table    I32 [B, max_pages], required for PA_BBND
+ *   out     same shape/dtype as q (written for every q row; rows with no
+ *           selected key get 0)
+ *   lse     F32, BNSD [B,N1,Sq] / TND [Tq,N1]; required when return_lse
+ *           (rows with no selected key get -inf)
+ */
+bsa_status bsa_fwd_get_workspace(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                                 const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
+                                 const bsa_tensor *cu_seqlens_kv, const bsa_tensor *seqused_kv,
+                                 const bsa_tensor *block_table, const bsa_params *params,
+                                 const bsa_tensor *out, const bsa_tensor *lse,
+                                 size_t *workspace_bytes);
+
+/* Same arguments, then the workspace and a cudaStream_t (NULL = legacy
+ * default stream).  Asynchronous: returns after the launches. */
+bsa_status bsa_fwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                   const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
+                   const bsa_tensor *cu_seqlens_kv, const bsa_tensor *seqused_kv,
+                   const bsa_tensor *block_table, const bsa_params *params,
+                   const bsa_tensor *out, const bsa_tensor *lse, void *workspace,
+                   size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------ backward */
+/* q, k, v, index, cu_seqlens_*, seqused_kv, block_table: as for bsa_fwd.
+ *   out, lse  the forward's outputs (lse required)
+ *   dout      same shape/dtype as q
+ *   dq        same shape/dtype as q; every row written
+ *   dk, dv    same shape/dtype as k / v.  Every kv row of every batch is
+ *             written (zeros where no query selects it), except that under
+ *             PA_BBND only the pages block_table[b][0 .. ceil(kvlen_b/page))
+ *             are written; other pages are left untouched.
+ */
+bsa_status bsa_bwd_get_workspace(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                                 const bsa_tensor *out, const bsa_tensor *dout,
+                                 const bsa_tensor *lse, const bsa_tensor *index,
+                                 const bsa_tensor *cu_seqlens_q, const bsa_tensor *cu_seqlens_kv,
+                                 const bsa_tensor *seqused_kv, const bsa_tensor *block_table,
+                                 const bsa_params *params, const bsa_tensor *dq,
+                                 const bsa_tensor *dk, const bsa_tensor *dv,
+                                 size_t *workspace_bytes);
+
+bsa_status bsa_bwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                   const bsa_tensor *out, const bsa_tensor *dout, const bsa_tensor *lse,
+                   const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
+                   const bsa_tensor *cu_seqlens_kv, const bsa_tensor *seqused_kv,
+                   const bsa_tensor *block_table, const bsa_params *params,
+                   const bsa_tensor *dq, const bsa_tensor *dk, const bsa_tensor *dv,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* ----------------------------------------------------- status, layout */
+/* Synchronises `stream`, then copies the workspace's status word (the
+ * BSA_FLAG_* bits raised by the last call that used this workspace). */
+bsa_status bsa_read_status(const void *workspace, void *stream, uint32_t *flags);
+
+const char *bsa_status_string(bsa_status status);
+
+/* Where the builders' results sit inside a workspace, so that callers (and
+ * the tests) can inspect them after a call.  Offsets are bytes from the
+ * workspace start; unused regions have bytes == 0.
+ *   status     uint32[16]: [0] flags, [2] forward items, [4] backward items,
+ *              [5] total kv blocks TK, [6] inverse-index entries
+ *   batch      per batch 12 x int32: qlen, kvlen, nq, nk, qoff, koff,
+ *              q_tok0 (2 words, int64), kv_tok0 (2 words, int64), kvst (kv
+ *              rows stored for the batch), 1 spare
+ *   comp       uint16 [Hidx][Rg][W] compacted index rows (0xFFFF padded)
+ *   ncomp      int32 [Hidx][Rg] accepted entries per row
+ *   fwd_items  int32 forward item ids in execution order
+ *   inv_off    int32 [Hidx*TK+1] CSR offsets of the KV-major inverse
+ *   inv_list   int32 batch-local query blocks per (index head, kv block)
+ *   bwd_items  int32 backward item ids in execution order
+ * Item ids: forward (h1*Rg + gq)*(BQ/128) + q_slice, gq the global query
+ * block row; backward (h2*TK + gk)*(BKV/128) + kv_slice, gk the global kv
+ * block (batch b's blocks after those of every earlier batch) and TK the
+ * total kv blocks of this call (status word [5]). */
+typedef struct bsa_ws_region {
+  uint64_t offset;
+  uint64_t bytes;
+} bsa_ws_region;
+
+typedef struct bsa_ws_layout {
+  bsa_ws_region status, batch, comp, ncomp, fwd_items, inv_off, inv_list, bwd_items;
+  bsa_ws_region dsum, dq_acc, sort_keys;
+  int64_t Rg;      /* global query-block rows (TND: R; BNSD: B*ceil(Sq/BQ)) */
+  int64_t tk_max;  /* upper bound on total kv blocks, from shapes */
+  uint64_t total_bytes;
+} bsa_ws_layout;
+
+bsa_status bsa_fwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                                    const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
+                                    const bsa_tensor *cu_seqlens_kv, const bsa_tensor *seqused_kv,
+                                    const bsa_tensor *block_table, const bsa_params *params,
+                                    const bsa_tensor *out, const bsa_tensor *lse,
+                                    bsa_ws_layout *layout);
+
+bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                                    const bsa_tensor *out, const bsa_tensor *dout,
+                                    const bsa_tensor *lse, const bsa_tensor *index,
+                                    const bsa_tensor *cu_seqlens_q,
+                                    const bsa_tensor *cu_seqlens_kv,
+                                    const bsa_tensor *seqused_kv, const bsa_tensor *block_table,
+                                    const bsa_params *params, const bsa_tensor *dq,
+                                    const bsa_tensor *dk, const bsa_tensor *dv,
+                                    bsa_ws_layout *layout);
+
+/* Library ABI version (bumped on any signature or layout change). */
+int32_t bsa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H_ */

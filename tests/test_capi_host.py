@@ -1,0 +1,154 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point the
+header declares, and its host-side validation and workspace sizing behave
+(these paths never touch device memory, so host tensors stand in)."""
+import os
+import re
+
+import pytest
+import torch
+
+import block_sparse_variable_b200 as bsa
+from workloads.gen import make_problem, pat_random_k
+from tests.harness import params_of
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:bsa_status|const char \*|int32_t)\s*(bsa_\w+)\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol():
+    names = _declared()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(bsa.lib(), n), n
+    assert set(names) == set(bsa.EXPORTED)
+    assert bsa.lib().bsa_abi_version() == 1
+
+
+def test_status_strings():
+    for code, name in bsa.STATUS_NAMES.items():
+        assert bsa.bsa_status_string(code).startswith(name)
+
+
+def _prob(**kw):
+    base = dict(layout_q="TND", layout_kv="TND", B=2, N1=4, N2=2, D=64, lens_q=[200, 130],
+                pattern=pat_random_k, seed_base=1)
+    base.update(kw)
+    return make_problem(**base)
+
+
+def _ws(p, params=None, **over):
+    a = dict(q=p.q, k=p.k, v=p.v, index=p.index, cu_seqlens_q=p.cu_q, cu_seqlens_kv=p.cu_kv,
+             seqused_kv=p.seqused_kv, block_table=p.block_table)
+    a.update(over)
+    return bsa.bsa_fwd_get_workspace(a.pop("q"), a.pop("k"), a.pop("v"), a.pop("index"),
+                                     params or params_of(p), **a)
+
+
+def _code(fn):
+    with pytest.raises(bsa.BsaError) as e:
+        fn()
+    return e.value.status
+
+
+def test_valid_layouts_size_workspace():
+    for kw in (dict(), dict(layout_q="BNSD", layout_kv="BNSD", Sq=300, lens_q=None, lens_kv=None),
+               dict(layout_kv="PA_BBND", page_size=256)):
+        p = _prob(**kw)
+        n = _ws(p)
+        lay = bsa.bsa_fwd_workspace_layout(p.q, p.k, p.v, p.index, params_of(p), cu_seqlens_q=p.cu_q,
+                                           cu_seqlens_kv=p.cu_kv, seqused_kv=p.seqused_kv,
+                                           block_table=p.block_table,
+                                           lse=torch.empty(p.q.shape[:-1] if p.layout_q == "TND"
+                                                           else p.q.shape[:-1], dtype=torch.float32))
+        assert n == lay.total_bytes > 0
+        regs = sorted((getattr(lay, f).offset, getattr(lay, f).bytes) for f in
+                      ("status", "batch", "comp", "ncomp", "fwd_items", "sort_keys")
+                      if getattr(lay, f).bytes)
+        for (o1, b1), (o2, _) in zip(regs, regs[1:]):
+            assert o1 + b1 <= o2 and o1 % 256 == 0
+        assert regs[-1][0] + regs[-1][1] <= n
+        assert lay.status.offset == 0
+
+
+def test_backward_workspace_has_inverse_and_accumulator():
+    p = _prob()
+    lse = torch.empty(p.q.shape[0], p.N1)
+    lay = bsa.bsa_bwd_workspace_layout(p.q, p.k, p.v, p.q, p.dout, lse, p.index, params_of(p),
+                                       cu_seqlens_q=p.cu_q, cu_seqlens_kv=p.cu_kv)
+    assert lay.inv_off.bytes and lay.inv_list.bytes and lay.bwd_items.bytes
+    assert lay.dq_acc.bytes == p.q.shape[0] * p.N1 * p.D * 4
+    assert lay.dsum.bytes == p.q.shape[0] * p.N1 * 4
+    n = bsa.bsa_bwd_get_workspace(p.q, p.k, p.v, p.q, p.dout, lse, p.index, params_of(p),
+                                  cu_seqlens_q=p.cu_q, cu_seqlens_kv=p.cu_kv)
+    assert n == lay.total_bytes
+
+
+def test_rejections():
+    p = _prob()
+    P = params_of(p)
+    ok = _ws(p)
+    assert ok > 0
+    # missing required pieces
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(p.q, p.k, p.v, p.index, P, cu_seqlens_kv=p.cu_kv)) \
+        == 161001
+    assert _code(lambda: _ws(p, cu_seqlens_kv=None)) == 161001
+    # shapes / dtypes / attributes
+    assert _code(lambda: _ws(p, k=p.k.float())) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "TND", 4, 3, (128, 128)))) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "TND", 4, 2, (64, 128)))) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "TND", 4, 2, (128, 2048)))) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "BNSD", 4, 2, (128, 128)))) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "TND", 5, 2, (128, 128)))) == 161002
+    assert _code(lambda: _ws(p, params=bsa.params_for("TND", "TND", 4, 2, (128, 128), scale=-1.0))) \
+        == 161002
+    assert _code(lambda: _ws(p, index=p.index.view(torch.int16))) == 161002
+    assert _code(lambda: _ws(p, index=p.index[:3])) == 161002          # Hidx not N1 / N2
+    assert _code(lambda: _ws(p, q=p.q[:, :, :48].contiguous(), k=p.k[:, :, :48].contiguous(),
+                             v=p.v[:, :, :48].contiguous())) == 161003   # D = 48
+    # strides: last dim contiguous, others 16-byte multiples
+    strided = torch.zeros(p.q.shape[0], p.q.shape[1], 128, dtype=p.q.dtype)[..., ::2]
+    assert _code(lambda: _ws(p, q=strided)) == 161002
+    wide = torch.zeros(p.q.shape[0], p.q.shape[1], 68, dtype=p.q.dtype)[..., :64]  # row stride 68
+    assert _code(lambda: _ws(p, q=wide)) == 161002
+    # paged: page size multiple of 128; seqused required
+    pp = _prob(layout_kv="PA_BBND", page_size=128)
+    assert _ws(pp) > 0
+    assert _code(lambda: _ws(pp, seqused_kv=None)) == 161001
+    assert _code(lambda: _ws(pp, cu_seqlens_kv=torch.zeros(3, dtype=torch.int64))) == 161002
+    p64 = _prob(layout_kv="PA_BBND", page_size=64)
+    assert _code(lambda: _ws(p64)) == 161003
+
+
+def test_bnsd_index_shape_and_lse():
+    p = _prob(layout_q="BNSD", layout_kv="BNSD", Sq=300, lens_q=None, lens_kv=None)
+    assert _ws(p) > 0
+    assert _code(lambda: _ws(p, index=p.index[:, :, :2])) == 161002     # rows != ceil(S/BQ)
+    P = params_of(p)
+    bad_lse = torch.empty(1, 4, 300)
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(p.q, p.k, p.v, p.index, P, lse=bad_lse)) == 161002
+
+
+def test_exec_rejects_small_workspace_before_any_launch():
+    p = _prob()
+    n = _ws(p)
+    ws = torch.zeros(n // 2, dtype=torch.uint8)
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_fwd(p.q, p.k, p.v, p.index, params_of(p), cu_seqlens_q=p.cu_q,
+                    cu_seqlens_kv=p.cu_kv, out=torch.empty_like(p.q),
+                    lse=torch.empty(p.q.shape[0], p.N1), workspace=ws, stream=0)
+    assert e.value.status == 161004
+
+
+def test_empty_query_is_a_no_op():
+    p = _prob()
+    q0 = p.q[:0]
+    cu = torch.zeros(3, dtype=torch.int64)
+    out, lse, _ = bsa.bsa_fwd(q0, p.k, p.v, p.index[:, :0], params_of(p), cu_seqlens_q=cu,
+                              cu_seqlens_kv=p.cu_kv, out=torch.empty_like(q0),
+                              lse=torch.empty(0, p.N1), workspace=torch.zeros(256, dtype=torch.uint8),
+                              stream=0)
+    assert out.numel() == 0

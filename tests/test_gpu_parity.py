@@ -1,0 +1,256 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Builders (compacted rows, inverse index, work lists,
+status flags) must match exactly; out/dq/dk/dv within max-abs 2e-2 and
+rel-L2 1e-2; lse within 1e-3.  Backward inputs are the oracle's out rounded
+to the input dtype and its lse in fp32, given to both sides."""
+import math
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_variable_b200 as bsa
+import oracle
+import workloads
+from oracle import builders
+from workloads.gen import (make_problem, pat_dense, pat_density, pat_fraction_diag, pat_random_k,
+                           pat_topk)
+from tests import harness as H
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "bnsd_random": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=2, D=64, Sq=384,
+                        pattern=pat_random_k),
+    "bnsd_ragged_kv": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=1, D=64, Sq=300,
+                           lens_kv=[300, 170], Skv=300, pattern=pat_density(0.5, 1)),
+    "bnsd_blocks_256x128": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=128,
+                                Sq=640, BQ=256, BKV=128, pattern=pat_density(0.4, 1)),
+    "bnsd_fp16_d128": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=3, N2=1, D=128, Sq=520,
+                           dtype=torch.float16, pattern=pat_random_k),
+    "tnd_gqa": dict(layout_q="TND", layout_kv="TND", B=3, N1=4, N2=2, D=64,
+                    lens_q=[130, 300, 77], lens_kv=[200, 129, 256], pattern=pat_fraction_diag(0.5)),
+    "tnd_gqa_d128": dict(layout_q="TND", layout_kv="TND", B=2, N1=8, N2=2, D=128,
+                         lens_q=[600, 257], lens_kv=[600, 257], pattern=pat_fraction_diag(0.25)),
+    "tnd_shared_rows": dict(layout_q="TND", layout_kv="TND", B=2, N1=4, N2=2, Hidx=2, D=64,
+                            lens_q=[256, 140], lens_kv=[256, 140], pattern=pat_random_k),
+    "tnd_seqused": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=2, D=64,
+                        lens_q=[200, 90], lens_kv=[150, 60], kv_storage=[260, 100],
+                        pattern=pat_random_k),
+    "tnd_empty_batches": dict(layout_q="TND", layout_kv="TND", B=3, N1=2, N2=2, D=64,
+                              lens_q=[0, 150, 40], lens_kv=[100, 0, 300], pattern=pat_random_k),
+    "paged": dict(layout_q="TND", layout_kv="PA_BBND", B=3, N1=4, N2=2, D=64,
+                  lens_q=[300, 129, 64], lens_kv=[300, 129, 64], page_size=128, extra_pages=2,
+                  pattern=pat_topk(2)),
+    "paged_256": dict(layout_q="TND", layout_kv="PA_BBND", B=2, N1=2, N2=1, D=128,
+                      lens_q=[700, 130], lens_kv=[600, 300], page_size=256, extra_pages=1,
+                      dtype=torch.float16, pattern=pat_random_k),
+    "big_blocks": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=2, D=64, BQ=512, BKV=256,
+                       lens_q=[700, 300], lens_kv=[900, 300], pattern=pat_random_k),
+    "blocks_1024": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=64, Sq=1500,
+                        BQ=1024, BKV=1024, dtype=torch.float16, pattern=pat_random_k),
+    "dense_many_blocks": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=1, N2=1, D=128, Sq=1100,
+                              pattern=pat_dense),
+}
+
+
+def _hook_invalid(rng, b, hi, i, sel):
+    if i == 0 and hi == 0:
+        return [1, 0xFFFF, 1, 0, 3, 9]
+    return sel
+
+
+def _hook_empty(rng, b, hi, i, sel):
+    return [] if (i % 2 == 1) else sel
+
+
+EDGE = {
+    "invalid_entries": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=64, Sq=512, W=6,
+                            pattern=pat_random_k, row_hook=_hook_invalid),
+    "empty_rows": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=64,
+                       lens_q=[384, 200], lens_kv=[256, 300], pattern=pat_random_k,
+                       row_hook=_hook_empty),
+}
+
+
+def _problem(name):
+    spec = dict(SMALL.get(name) or EDGE[name])
+    return make_problem(seed_base=zlib.crc32(name.encode()) % 9973, name=name, **spec)
+
+
+def _oracle(p):
+    o = oracle.Oracle(p)
+    out, lse, fl = o.fwd()
+    out_b = out.to(p.dtype)
+    lse_f = lse.float()
+    dq, dk, dv, fl2 = o.bwd(out_b, p.dout, lse_f)
+    return dict(out=out, lse=lse, out_b=out_b, lse_f=lse_f, dq=dq, dk=dk, dv=dv,
+                flags=fl | fl2 | o.scan_flags())
+
+
+def _check_builders(p, ws_f, ws_b, lay_f, lay_b, B):
+    st_f = H.region(ws_f, lay_f.status, torch.int32).astype(np.int64)
+    st_b = H.region(ws_b, lay_b.status, torch.int32).astype(np.int64)
+    geo = B["geo"]
+    assert st_f[0] == B["flags"] and st_b[0] == B["flags"]
+    assert st_f[5] == geo.TK and st_b[5] == geo.TK
+    n_f = int(st_f[2])
+    assert n_f == len(B["fwd_items"])
+    Hidx, Rg, W = p.Hidx, geo.Rg, p.W
+    comp = H.region(ws_f, lay_f.comp, torch.int16).view(np.uint16).reshape(Hidx, Rg, W)
+    ncomp = H.region(ws_f, lay_f.ncomp, torch.int32).reshape(Hidx, Rg)
+    assert np.array_equal(ncomp, B["ncomp"])
+    assert np.array_equal(comp, B["comp"])
+    assert np.array_equal(H.region(ws_f, lay_f.fwd_items, torch.int32, n_f), B["fwd_items"])
+    nnz = int(st_b[6])
+    off = H.region(ws_b, lay_b.inv_off, torch.int32, Hidx * geo.TK + 1)
+    assert np.array_equal(off, B["inv_off"]) and nnz == len(B["inv_list"])
+    assert np.array_equal(H.region(ws_b, lay_b.inv_list, torch.int32, nnz), B["inv_list"])
+    n_b = int(st_b[4])
+    assert n_b == len(B["bwd_items"])
+    assert np.array_equal(H.region(ws_b, lay_b.bwd_items, torch.int32, n_b), B["bwd_items"])
+
+
+def _run_and_check(p):
+    R = _oracle(p)
+    Bld = builders.build_all(p)
+    d = H.device_inputs(p)
+    out, lse, ws_f, _ = H.gpu_fwd(p, d)
+    torch.cuda.synchronize()
+    H.check_close("out", out, R["out"])
+    H.check_lse(lse, R["lse"])
+    # backward on the oracle's (rounded) forward results; sentinel-filled outputs
+    dk0 = torch.full_like(d["k"], float("nan"))
+    dv0 = torch.full_like(d["v"], float("nan"))
+    dq0 = torch.full_like(d["q"], float("nan"))
+    dq, dk, dv, ws_b, _ = H.gpu_bwd(p, R["out_b"].cuda(), R["lse_f"].cuda(), d, dq=dq0, dk=dk0, dv=dv0)
+    torch.cuda.synchronize()
+    wm = H.kv_written_mask(p)
+    qmask = None
+    if p.layout_q == "TND":
+        qmask = torch.zeros(p.q.shape[:-1], dtype=torch.bool)
+        qmask[:int(p.cu_q[-1])] = True
+    H.check_close("dq", dq, R["dq"], qmask)
+    H.check_close("dk", dk, R["dk"], wm)
+    H.check_close("dv", dv, R["dv"], wm)
+    if (~wm).any():   # rows the backward must leave alone stay untouched
+        assert torch.isnan(dk.cpu()[~wm]).all() and torch.isnan(dv.cpu()[~wm]).all()
+    lay_f = bsa.bsa_fwd_workspace_layout(d["q"], d["k"], d["v"], d["index"], H.params_of(p),
+                                         lse=lse, **H.opt_kwargs(d))
+    lay_b = bsa.bsa_bwd_workspace_layout(d["q"], d["k"], d["v"], out, d["dout"], lse, d["index"],
+                                         H.params_of(p), **H.opt_kwargs(d))
+    _check_builders(p, ws_f, ws_b, lay_f, lay_b, Bld)
+    assert bsa.bsa_read_status(ws_f) == R["flags"]
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_cases(name):
+    _run_and_check(_problem(name))
+
+
+@pytest.mark.parametrize("name", sorted(EDGE))
+def test_edge_cases(name):
+    _run_and_check(_problem(name))
+
+
+@pytest.mark.parametrize("c", [1, 2])
+def test_configs_full(c):
+    _run_and_check(workloads.make_config(c))
+
+
+def test_return_lse_off_and_repeat_calls():
+    """lse may be omitted; a reused workspace gives identical results."""
+    p = _problem("tnd_gqa")
+    d = H.device_inputs(p)
+    P = H.params_of(p, return_lse=False)
+    out1, lse1, ws = bsa.bsa_fwd(d["q"], d["k"], d["v"], d["index"], P, **H.opt_kwargs(d))
+    assert lse1 is None
+    out2, _, _ = bsa.bsa_fwd(d["q"], d["k"], d["v"], d["index"], P, workspace=ws, **H.opt_kwargs(d))
+    torch.cuda.synchronize()
+    assert torch.equal(out1, out2)
+
+
+def test_chain_gpu_forward_then_backward():
+    """GPU fwd -> GPU bwd against oracle fwd -> oracle bwd."""
+    p = _problem("tnd_gqa_d128")
+    o = oracle.Oracle(p)
+    out, lse, _ = o.fwd()
+    dq, dk, dv, _ = o.bwd(out, p.dout, lse)
+    g_out, g_lse, _, d = H.gpu_fwd(p)
+    g_dq, g_dk, g_dv, _, _ = H.gpu_bwd(p, g_out, g_lse, d)
+    torch.cuda.synchronize()
+    H.check_close("dq", g_dq, dq)
+    H.check_close("dk", g_dk, dk)
+    H.check_close("dv", g_dv, dv)
+
+
+# --------------------------------------------------------------- full sizes
+def _sample_q_rows(o, n, rng):
+    rows = o.q_rows_all()
+    pick = rng.choice(len(rows), size=min(n, len(rows)), replace=False)
+    return rows[np.sort(pick)]
+
+
+@pytest.mark.parametrize("c", [3, 4, 5])
+def test_configs_full_size_sampled(c):
+    """Full-size workloads, launched exactly as the benchmark does: builders
+    compared in full, outputs on sampled rows the oracle computes one by one.
+    The backward covers one kv-head group (its q heads get the oracle's
+    forward as out/lse; other heads get out 0 and lse +inf, so they add
+    nothing), sampled dq rows of the group and sampled dk/dv rows."""
+    p = workloads.make_config(c)
+    o = oracle.Oracle(p)
+    rng = np.random.default_rng(c)
+    d = H.device_inputs(p)
+    out, lse, ws_f, _ = H.gpu_fwd(p, d)
+    torch.cuda.synchronize()
+    rows = _sample_q_rows(o, 96, rng)
+    r_out, r_lse, fl = o.fwd_rows(rows)
+    H.check_close("out(sampled)", o.gather_q(out.cpu(), rows), torch.from_numpy(r_out))
+    H.check_lse(o.gather_q(lse.cpu(), rows), torch.from_numpy(r_lse))
+
+    # builders in full
+    Bld = builders.build_all(p)
+    lay_f = bsa.bsa_fwd_workspace_layout(d["q"], d["k"], d["v"], d["index"], H.params_of(p),
+                                         lse=lse, **H.opt_kwargs(d))
+    st = H.region(ws_f, lay_f.status, torch.int32)
+    assert st[0] == Bld["flags"] == 0
+    n_f = int(st[2])
+    assert np.array_equal(H.region(ws_f, lay_f.fwd_items, torch.int32, n_f), Bld["fwd_items"])
+
+    # backward on one kv-head group
+    h2 = int(rng.integers(0, p.N2))
+    g = p.N1 // p.N2
+    b_sel = int(rng.integers(0, p.B)) if p.layout_q == "BNSD" else None
+    all_rows = o.q_rows_all()
+    grp = (all_rows[:, 1] // g) == h2
+    if b_sel is not None:
+        grp &= all_rows[:, 0] == b_sel
+    grows = all_rows[grp]
+    g_out, g_lse, _ = o.fwd_rows(grows)
+    out_in = torch.zeros(p.q.shape, dtype=p.dtype)
+    lse_in = torch.full(o.lse_shape(), float("inf"), dtype=torch.float32)
+    o._scatter_q(out_in, grows, torch.from_numpy(g_out).to(p.dtype))
+    o._scatter_stat(lse_in, grows, torch.from_numpy(g_lse).float())
+    dq, dk, dv, ws_b, _ = H.gpu_bwd(p, out_in.cuda(), lse_in.cuda(), d)
+    torch.cuda.synchronize()
+    qs = grows[np.sort(rng.choice(len(grows), size=min(64, len(grows)), replace=False))]
+    r_dq, _ = o.bwd_dq_rows(out_in, p.dout, lse_in, qs)
+    H.check_close("dq(sampled)", o.gather_q(dq.cpu(), qs), torch.from_numpy(r_dq))
+    kvr = o.kv_rows_all()
+    kvr = kvr[kvr[:, 1] == h2]
+    if b_sel is not None:
+        kvr = kvr[kvr[:, 0] == b_sel]
+    ks = kvr[np.sort(rng.choice(len(kvr), size=min(64, len(kvr)), replace=False))]
+    r_dk, r_dv, _ = o.bwd_dkv_rows(out_in, p.dout, lse_in, ks)
+    ix = o.kv_index(ks)
+    H.check_close("dk(sampled)", dk.cpu()[ix], torch.from_numpy(r_dk))
+    H.check_close("dv(sampled)", dv.cpu()[ix], torch.from_numpy(r_dv))
+    lay_b = bsa.bsa_bwd_workspace_layout(d["q"], d["k"], d["v"], out, d["dout"], lse, d["index"],
+                                         H.params_of(p), **H.opt_kwargs(d))
+    stb = H.region(ws_b, lay_b.status, torch.int32)
+    assert stb[4] == len(Bld["bwd_items"])
+    assert np.array_equal(H.region(ws_b, lay_b.bwd_items, torch.int32, int(stb[4])), Bld["bwd_items"])
+    nnz = int(stb[6])
+    assert np.array_equal(H.region(ws_b, lay_b.inv_list, torch.int32, nnz), Bld["inv_list"])
