@@ -223,7 +223,7 @@ def bsa_fwd(q, k, v, index, params: Params, *, cu_seqlens_q=None, cu_seqlens_kv=
     n = ctypes.c_size_t(0)
     _check(_lib.bsa_fwd_get_workspace(*[_ref(x) for x in ins], ctypes.byref(cp), _ref(o), _ref(l),
                                       ctypes.byref(n)), "bsa_fwd_get_workspace")
-    if workspace is None or workspace.numel() < n.value:
+    if workspace is None:
         workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=q.device)
     _check(_lib.bsa_fwd(*[_ref(x) for x in ins], ctypes.byref(cp), _ref(o), _ref(l),
                         ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()),
@@ -278,7 +278,7 @@ def bsa_bwd(q, k, v, out, dout, lse, index, params: Params, *, cu_seqlens_q=None
     _check(_lib.bsa_bwd_get_workspace(*[_ref(x) for x in ins], ctypes.byref(cp),
                                       *[_ref(x) for x in outs], ctypes.byref(n)),
            "bsa_bwd_get_workspace")
-    if workspace is None or workspace.numel() < n.value:
+    if workspace is None:
         workspace = torch.empty(max(n.value, 256), dtype=torch.uint8, device=q.device)
     _check(_lib.bsa_bwd(*[_ref(x) for x in ins], ctypes.byref(cp), *[_ref(x) for x in outs],
                         ctypes.c_void_p(workspace.data_ptr()), ctypes.c_size_t(workspace.numel()),
