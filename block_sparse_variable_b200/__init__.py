@@ -90,7 +90,7 @@ _lib = _load()
 
 EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bwd",
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
-            "bsa_bwd_workspace_layout", "bsa_abi_version")
+            "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace")
 
 
 def lib():
@@ -296,3 +296,35 @@ def bsa_read_status(workspace: torch.Tensor, stream=None) -> int:
 
 def bsa_status_string(status: int) -> str:
     return _lib.bsa_status_string(int(status)).decode()
+
+
+# ------------------------------------------------- forward without workspace
+STATIC_WORKSPACE_BYTES = 32 << 20
+
+
+def bsa_fwd_static_workspace(q, k, v, index, params: Params, *, cu_seqlens_q=None,
+                             cu_seqlens_kv=None, seqused_kv=None, block_table=None, out=None,
+                             lse=None, stream=None):
+    """Forward for callers that cannot allocate device memory at run time.
+
+    The library's built-in 32 MiB scratch array replaces the workspace, so
+    the call allocates nothing (``out`` / ``lse`` must then be passed in by
+    such a caller; they are only created here for convenience when None).
+    Calls that may overlap on the GPU share the array and must be
+    serialised by the caller.  Returns (out, lse).
+    """
+    f = _lib.bsa_fwd_static_workspace
+    if f.argtypes is None:
+        T = ctypes.POINTER(bsa_tensor)
+        f.argtypes = [T] * 8 + [ctypes.POINTER(bsa_params), T, T, ctypes.c_void_p]
+        f.restype = ctypes.c_int
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and params.return_lse:
+        lse = torch.empty(_lse_shape(q, params), dtype=torch.float32, device=q.device)
+    ins, o, l = _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table,
+                           out, lse)
+    cp = params.c()
+    _check(f(*[_ref(x) for x in ins], ctypes.byref(cp), _ref(o), _ref(l),
+             ctypes.c_void_p(_stream(stream))), "bsa_fwd_static_workspace")
+    return out, lse

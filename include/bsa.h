@@ -142,6 +142,34 @@ bsa_status bsa_fwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
                    const bsa_tensor *out, const bsa_tensor *lse, void *workspace,
                    size_t workspace_bytes, void *stream);
 
+/* Forward without a caller-supplied workspace; allocates nothing.
+ * (An addition of this library: the pages have no counterpart.)
+ *
+ * For callers that cannot allocate device memory when they run the
+ * forward -- for example a plugin executed by an inference runtime whose
+ * contract forbids allocation inside its execute step, or an engine that
+ * fixes its device-memory budget at start-up.  Arguments and results are
+ * those of bsa_fwd; the caller still passes every input and output.  The
+ * scratch lives in a fixed 32 MiB array inside the library that every GPU
+ * loading the library keeps until the process exits.
+ *   - A problem whose forward workspace (bsa_fwd_get_workspace) exceeds
+ *     32 MiB is rejected with BSA_ERR_WORKSPACE before any launch.
+ *   - The first call on a device looks up the array's device address
+ *     (a CUDA runtime query) and caches it; make that first call before any
+ *     stream capture on that device.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     each call initialises everything it reads, but two calls that may
+ *     overlap on the GPU (different streams, different threads) race and
+ *     must be serialised by the caller.
+ *   - bsa_read_status cannot see this scratch; the status word is not
+ *     available to the caller. */
+bsa_status bsa_fwd_static_workspace(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
+                                    const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
+                                    const bsa_tensor *cu_seqlens_kv,
+                                    const bsa_tensor *seqused_kv, const bsa_tensor *block_table,
+                                    const bsa_params *params, const bsa_tensor *out,
+                                    const bsa_tensor *lse, void *stream);
+
 /* ------------------------------------------------------------ backward */
 /* q, k, v, index, cu_seqlens_*, seqused_kv, block_table: as for bsa_fwd.
  *   out, lse  the forward's outputs (lse required)

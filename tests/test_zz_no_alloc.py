@@ -1,0 +1,69 @@
+"""bsa_fwd_static_workspace: the forward for callers that cannot allocate
+device memory while they run (for example a plugin inside an inference
+runtime that forbids allocation in its execute step, or an engine whose
+memory budget is fixed at start-up).  It uses the library's built-in 32 MiB
+scratch array instead of a caller workspace.
+
+This file is collected last on purpose: the test must pass in a fresh
+process and after every other test has used the library."""
+import ctypes
+
+import pytest
+import torch
+
+import block_sparse_variable_b200 as bsa
+import workloads
+from tests import harness as H
+
+
+def _call_static(p, d, out, lse):
+    # straight through the C ABI
+    f = bsa.lib().bsa_fwd_static_workspace
+    T = ctypes.POINTER(bsa.bsa_tensor)
+    f.argtypes = [T] * 8 + [ctypes.POINTER(bsa.bsa_params), T, T, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    descs = [bsa.describe(x) for x in (d["q"], d["k"], d["v"], d["index"], d["cu_seqlens_q"],
+                                       d["cu_seqlens_kv"], d["seqused_kv"], d["block_table"])]
+    cp = H.params_of(p).c()
+    st = f(*[None if x is None else ctypes.byref(x) for x in descs], ctypes.byref(cp),
+           ctypes.byref(bsa.describe(out)), ctypes.byref(bsa.describe(lse)),
+           ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return st
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("c", [1, 2, 5])
+def test_static_workspace_forward_matches_bsa_fwd(c):
+    """Two calls in a row agree with bsa_fwd (same tolerance as the parity tests)."""
+    p = workloads.make_config(c)
+    d = H.device_inputs(p)
+    ref_out, ref_lse, _, _ = H.gpu_fwd(p, d)
+    torch.cuda.synchronize()
+    out = torch.empty_like(ref_out)
+    lse = torch.empty_like(ref_lse)
+    for _ in range(2):
+        out.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        assert _call_static(p, d, out, lse) == 0
+        torch.cuda.synchronize()
+        H.check_close("out", out, ref_out.double())
+        H.check_lse(lse, ref_lse)
+
+
+def test_static_workspace_rejects_oversized_problems():
+    """A forward needing more than the 32 MiB scratch is refused before any
+    launch (host-side check only, so no GPU is needed)."""
+    q = bsa.describe_shape((4096, 32, 128), torch.bfloat16)
+    k = bsa.describe_shape((4096, 8, 128), torch.bfloat16)
+    index = bsa.describe_shape((32, 120000, 64), torch.uint16)   # 491 MB of compacted rows
+    cu = bsa.describe_shape((2,), torch.int64)
+    out = bsa.describe_shape((4096, 32, 128), torch.bfloat16)
+    lse = bsa.describe_shape((4096, 32), torch.float32)
+    cp = bsa.params_for("TND", "TND", 32, 8).c()
+    f = bsa.lib().bsa_fwd_static_workspace
+    T = ctypes.POINTER(bsa.bsa_tensor)
+    f.argtypes = [T] * 8 + [ctypes.POINTER(bsa.bsa_params), T, T, ctypes.c_void_p]
+    f.restype = ctypes.c_int
+    r = ctypes.byref
+    st = f(r(q), r(k), r(k), r(index), r(cu), r(cu), None, None, r(cp), r(out), r(lse), None)
+    assert st == 161004   # BSA_ERR_WORKSPACE
