@@ -1,0 +1,79 @@
+// tma_maps.cu -- encodes the TMA tensor maps of one call (host side).  The
+// driver's cuTensorMapEncodeTiled is reached through the runtime's
+// entry-point query, so the library needs no link-time libcuda.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "tc_common.h"
+
+namespace bsa {
+namespace {
+
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiled encoder() {
+  static EncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiled>(f);
+  });
+  return fn;
+}
+
+cudaError_t encode(CUtensorMap *m, const Problem &p, const void *base, const cuuint64_t dims[4],
+                   const cuuint64_t strides[3], const cuuint32_t box[4]) {
+  EncodeTiled fn = encoder();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  const CUtensorMapDataType dt =
+      p.dtype == BSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUresult r = fn(m, dt, 4, const_cast<void *>(base), dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cuuint64_t nz(int64_t x) { return x > 0 ? cuuint64_t(x) : 16; }
+
+cudaError_t kv_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb, int64_t sh,
+                   int64_t st) {
+  const cuuint64_t D = cuuint64_t(p.D);
+  if (p.kv_layout == BSA_LAYOUT_PA_BBND) {
+    const cuuint64_t dims[4] = {D, cuuint64_t(p.N2), cuuint64_t(p.page_size), cuuint64_t(p.num_pages)};
+    const cuuint64_t strides[3] = {nz(sh * 2), nz(st * 2), nz(sb * 2)};
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    return encode(m, p, base, dims, strides, box);
+  }
+  const int64_t rows = p.kv_layout == BSA_LAYOUT_TND ? p.Tkv : p.Skv;
+  const int64_t nb = p.kv_layout == BSA_LAYOUT_TND ? 1 : p.B;
+  const cuuint64_t dims[4] = {D, cuuint64_t(rows), cuuint64_t(p.N2), cuuint64_t(nb)};
+  const cuuint64_t strides[3] = {nz(st * 2), nz(sh * 2), nz(p.kv_layout == BSA_LAYOUT_TND ? rows * st * 2 : sb * 2)};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  return encode(m, p, base, dims, strides, box);
+}
+
+}  // namespace
+
+cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m) {
+  const int64_t rows = p.q_layout == BSA_LAYOUT_TND ? p.Tq : p.Sq;
+  const int64_t nb = p.q_layout == BSA_LAYOUT_TND ? 1 : p.B;
+  const cuuint64_t dims[4] = {cuuint64_t(p.D), cuuint64_t(rows), cuuint64_t(p.N1), cuuint64_t(nb)};
+  const cuuint64_t strides[3] = {nz(p.q_st * 2), nz(p.q_sh * 2),
+                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * p.q_st * 2 : p.q_sb * 2)};
+  const cuuint32_t box[4] = {64, 128, 1, 1};
+  cudaError_t e = encode(&m.q, p, p.q, dims, strides, box);
+  if (e != cudaSuccess) return e;
+  if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
+  return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);
+}
+
+}  // namespace bsa
