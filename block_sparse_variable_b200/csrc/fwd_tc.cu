@@ -40,7 +40,7 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 384;
 constexpr int kStages = 2;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: any legitimate wait is far shorter
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows by > 2^8
@@ -68,7 +68,8 @@ struct Layout {
   static constexpr int kK = kQ + kTile;
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBars = kV + kStages * kTile;
-  static constexpr int kTmemPtr = kBars + kNumBars * 8;
+  static constexpr int kXchg = kBars + kNumBars * 8 + 8;  // [2][2][128] floats (max, sum)
+  static constexpr int kTmemPtr = kXchg + 2 * 2 * 128 * 4;
   static constexpr int kAbort = kTmemPtr + 4;
   static constexpr int kBytes = kAbort + 4;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
@@ -164,6 +165,10 @@ __device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatil
   return __all_sync(0xffffffffu, r);
 }
 
+__device__ __forceinline__ void named_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
+}
+
 // drain wait on the abort path: bounded, result ignored
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
@@ -214,7 +219,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem, tO = tmem + 256;
+  const uint32_t tS0 = tmem, tO0 = tmem + 256;  // S_w at tS0 + 128w, O_w at tO0 + D*w
 
   if (warp == 0) {
     // ------------------------------------------------------ TMA producer
@@ -299,7 +304,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint64_t bdesc = sw128_desc(sV + s * L::kTile + kk * 2048, L::kBox, 1024);
-          mma_ts(tO, a_tmem + uint32_t(kk) * 8u, bdesc, idPV, (first && kk == 0) ? 0u : 1u);
+          mma_ts(tO0 + uint32_t(s) * D, a_tmem + uint32_t(kk) * 8u, bdesc, idPV,
+                 (first && kk == 0) ? 0u : 1u);
         }
         mma_commit(bar(kBarPVDone + s));
         mma_commit(bar(kBarVEmpty + s));
@@ -332,12 +338,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (j == n - 1) mma_commit(bar(kBarQEmpty));
         }
         __syncwarp();
-        if (j >= 1) issue_pv(kv_it - 1, j == 1, prev_valid);
+        if (j >= 1) issue_pv(kv_it - 1, j <= 2, prev_valid);
         prev_valid = v.kvlen - v.u0(ch);
         ch = next_chunk(p, v, ch);
         ++kv_it;
       }
-      if (ok) issue_pv(kv_it - 1, n == 1, prev_valid);
+      if (ok) issue_pv(kv_it - 1, n <= 2, prev_valid);
     }
     if (*abort && lane == 0) {  // let issued MMAs finish before TMEM is freed
       mma_commit(bar(kBarDrain));
@@ -345,114 +351,142 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     __syncwarp();
   } else if (warp >= 4) {
-    // ------------------------------------------------- softmax warpgroup
-    const int r = tid - 128;                       // query row = TMEM lane
-    const uint32_t lane_off = uint32_t((warp - 4) * 32) << 16;
+    // ------------------------------------------- two softmax warpgroups
+    // Warpgroup w takes the chunks whose global index t has t % 2 == w: its
+    // own S buffer, O accumulator, running max and sum (a split of the kv
+    // range inside the CTA); the halves are merged in the epilogue.
+    const int wg = (warp - 4) >> 2;
+    const int r = (tid - 128) & 127;                        // query row = TMEM lane
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    const uint32_t tS = tS0 + uint32_t(wg) * 128u + lane_off;
+    const uint32_t tOw = tO0 + uint32_t(wg) * D + lane_off;
+    float *xm = reinterpret_cast<float *>(sbase + L::kXchg);  // [2][128] max
+    float *xl = xm + 256;                                     // [2][128] sum
     const float kLn2 = 0.6931471805599453f;
-    uint32_t kv_it = 0;
+    uint32_t kv_it = 0, own = 0;  // global chunk counter; chunks this group took
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const ItemView v = item_view(p, p.fwd_items[it]);
-      T *orow = static_cast<T *>(p.out) + q_row(p.o_sb, p.o_sh, p.o_st, v.bi, v.b, v.h1, v.t0 + r);
-      float *lrow = p.lse ? p.lse + q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1, v.t0 + r) : nullptr;
       float m = -INFINITY, l = 0.f;
-      int j = 0;
-      for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok; ch = next_chunk(p, v, ch), ++j) {
-        const int s = int(kv_it % kStages);
-        const uint32_t ph = (kv_it / kStages) & 1u;
-        if (!(ok = wait_warp(bar(kBarSFull + s), ph, abort, p.status))) break;
+      int n = 0;
+      for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
+           ch = next_chunk(p, v, ch), ++n, ++kv_it) {
+        if (int(kv_it & 1u) != wg) continue;
+        if (!(ok = wait_warp(bar(kBarSFull + wg), own & 1u, abort, p.status))) break;
         tc_fence_after();
-        const uint32_t tS = tS0 + uint32_t(s) * 128u + lane_off;
-        uint32_t raw[4][32];
+        const int valid = v.kvlen - v.u0(ch);  // kv columns of this chunk that exist
+        // the whole 128-column row in one round trip
+        uint32_t x[4][32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + uint32_t(q) * 32u, raw[q]);
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + uint32_t(q) * 32u, x[q]);
         tmem_wait_ld();
-        const int u0 = v.u0(ch);
-        const int valid = v.kvlen - u0;  // kv columns of this chunk that exist
-        float mx = -INFINITY;
+        if (valid < 128) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (q * 32 + c >= valid) x[q][c] = __float_as_uint(-INFINITY);
+        }
+        float pm[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float x = __uint_as_float(raw[q][c]);
-            if (q * 32 + c >= valid) x = -INFINITY;
-            raw[q][c] = __float_as_uint(x);
-            mx = fmaxf(mx, x);
-          }
-        const float m_new = fmaxf(m, mx * p.scale_log2);
-        // first chunk: adopt the max (O is still empty); later chunks keep a
-        // stale max until it falls more than 2^8 behind (then P <= 256)
+          for (int c = 0; c < 32; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(x[q][c]));
+        const float cmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
+                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * p.scale_log2;
+        // running max: adopted on the group's first chunk; afterwards kept
+        // stale until it falls more than 2^8 behind (then O and l rescale)
         const bool first = m == -INFINITY;
-        const bool grow = !first && m_new > m + kRescaleThreshold;
-        if (first) m = m_new;
-        if (__any_sync(0xffffffffu, grow)) {
-          // O may only be rescaled once P_{j-1} V_{j-1} (and so every earlier
-          // product, the tensor pipe being in order) has landed in it
-          const uint32_t t = kv_it - 1;
-          if (!(ok = wait_warp(bar(kBarPVDone + int(t % 2)), (t / 2) & 1u, abort, p.status))) break;
+        const bool grow = __any_sync(0xffffffffu, !first && cmax > m + kRescaleThreshold);
+        const float m_new = first ? cmax : (grow ? fmaxf(m, cmax) : m);
+        const float alpha = (first || !grow) ? 1.f : ex2(m - m_new);
+        m = m_new;
+        // P = exp2(scale*log2(e)*s - m), written over S as 16-bit pairs
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int q = 0; q < 2; ++q)
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const float e0 = ex2(fmaf(__uint_as_float(x[2 * h + q][c]), p.scale_log2, -m));
+              const float e1 = ex2(fmaf(__uint_as_float(x[2 * h + q][c + 1]), p.scale_log2, -m));
+              ps[(c >> 1) & 3] += e0 + e1;
+              pk[q * 16 + (c >> 1)] = MmaOp<T>::pack(e0, e1);
+            }
+          tmem_st32(tS + uint32_t(h) * 32u, pk);
+        }
+        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
+        if (grow) {
+          // O may only be rescaled once this group's previous P V (t - 2,
+          // same accumulator) has landed in it
+          const uint32_t t = kv_it - 2;
+          if (!(ok = wait_warp(bar(kBarPVDone + wg), (t / 2) & 1u, abort, p.status))) break;
           tc_fence_after();
-          const float alpha = ex2(m - m_new);  // 1 for rows whose max did not grow
-          l *= alpha;
-          m = m_new;
 #pragma unroll
           for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
-            tmem_ld32(tO + lane_off + uint32_t(q) * 32u, o);
+            tmem_ld32(tOw + uint32_t(q) * 32u, o);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tO + lane_off + uint32_t(q) * 32u, o);
+            tmem_st32(tOw + uint32_t(q) * 32u, o);
           }
         }
-        const float basev = m == -INFINITY ? 0.f : m;
-        float rs = 0.f;
-        uint32_t pk[2][32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const float e0 = ex2(fmaf(__uint_as_float(raw[q][c]), p.scale_log2, -basev));
-            const float e1 = ex2(fmaf(__uint_as_float(raw[q][c + 1]), p.scale_log2, -basev));
-            rs += e0 + e1;
-            pk[q >> 1][(q & 1) * 16 + (c >> 1)] = MmaOp<T>::pack(e0, e1);
-          }
-        l += rs;
-        tmem_st32(tS + 0u, pk[0]);
-        tmem_st32(tS + 32u, pk[1]);
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(bar(kBarPFull + s));
-        ++kv_it;
+        mbar_arrive(bar(kBarPFull + wg));
+        ++own;
       }
       if (!ok) break;
-      // epilogue
+      // ---- epilogue: merge the two groups' partial results
       const bool live = r < v.rows;
-      if (j > 0) {
-        const uint32_t t = kv_it - 1;  // the item's last P V product
-        if (!(ok = wait_warp(bar(kBarPVDone + int(t % 2)), (t / 2) & 1u, abort, p.status))) break;
+      T *orow = static_cast<T *>(p.out) + q_row(p.o_sb, p.o_sh, p.o_st, v.bi, v.b, v.h1, v.t0 + r);
+      if (n > 0) {
+        const uint32_t t = kv_it - 1;  // the item's last P V; earlier ones precede it
+        if (!(ok = wait_warp(bar(kBarPVDone + int(t & 1u)), (t / 2) & 1u, abort, p.status))) break;
         tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-        for (int q = 0; q < D / 32; ++q) {
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + uint32_t(q) * 32u, o);
-          tmem_wait_ld();
-          if (live) {
-            uint4 w[4];
-            uint32_t *wp = reinterpret_cast<uint32_t *>(w);
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              wp[c] = MmaOp<T>::pack(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
-#pragma unroll
-            for (int c = 0; c < 4; ++c) reinterpret_cast<uint4 *>(orow + q * 32)[c] = w[c];
-          }
-        }
-        tc_fence_before();
-      } else if (live) {
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4 *>(orow)[c] = make_uint4(0, 0, 0, 0);
       }
-      if (live && lrow) *lrow = (l > 0.f) ? (m + __log2f(l)) * kLn2 : -INFINITY;
+      xm[wg * 128 + r] = m;
+      xl[wg * 128 + r] = l;
+      named_sync(1, 256);
+      const float m0 = xm[r], m1 = xm[128 + r], l0 = xl[r], l1 = xl[128 + r];
+      const float M = fmaxf(m0, m1);
+      const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
+      const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
+      const float Lsum = l0 * a0 + l1 * a1;
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      // group w writes columns [w*D/2, (w+1)*D/2) from both accumulators
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        const uint32_t col = uint32_t(wg) * (D / 2) + uint32_t(q) * 16u;
+        uint32_t o0[16], o1[16];
+        tmem_ld16(tO0 + lane_off + col, o0);
+        tmem_ld16(tO0 + uint32_t(D) + lane_off + col, o1);
+        tmem_wait_ld();
+        if (live) {
+          uint4 w[2];
+          uint32_t *wp = reinterpret_cast<uint32_t *>(w);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const float y0 = (a0 > 0.f ? __uint_as_float(o0[2 * c]) * a0 : 0.f) +
+                             (a1 > 0.f ? __uint_as_float(o1[2 * c]) * a1 : 0.f);
+            const float y1 = (a0 > 0.f ? __uint_as_float(o0[2 * c + 1]) * a0 : 0.f) +
+                             (a1 > 0.f ? __uint_as_float(o1[2 * c + 1]) * a1 : 0.f);
+            wp[c] = MmaOp<T>::pack(y0 * inv, y1 * inv);
+          }
+          reinterpret_cast<uint4 *>(orow + col)[0] = w[0];
+          reinterpret_cast<uint4 *>(orow + col)[1] = w[1];
+        }
+      }
+      if (wg == 0 && live && p.lse)
+        p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1, v.t0 + r)] =
+            Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+      tc_fence_before();
+      named_sync(1, 256);  // both groups are done with O and the exchange slots
     }
   }
   tc_fence_before();
