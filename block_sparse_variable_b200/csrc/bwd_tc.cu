@@ -1,0 +1,508 @@
+// bwd_tc.cu -- tcgen05 / TMEM / TMA backward main kernel for sm_100a.
+//
+// BlockSparseAttentionGrad README, "Formula", in the stage order of the
+// aclnnFlashAttentionUnpaddingScoreGradV2 article, section 8.3 (recompute p,
+// dp, ds, dq, dk, dv).  KV-major: one work item is a 128-row kv chunk of kv
+// head h2; its K and V stay in shared memory and dK, dV accumulate in TMEM
+// while the item walks, for every q head of the GQA group, the query blocks
+// that selected its kv block (the inverted index) in 128-row q steps:
+//   phase 1 (two interleaved MMA chains):
+//     S^T  = K Q^T          -> TMEM R0        (M = kv, N = q, K = D)
+//     dP^T = V dOut^T       -> TMEM R1
+//   softmax warps (thread = kv row, group w = q columns [64w, 64w+64)):
+//     P^T  = exp2(scale*log2(e)*S^T - lse*log2(e))   (0 for rows/cols outside)
+//     dS^T = P^T o (dP^T - Dsum)
+//     P and dS packed to 16-bit pairs into the group's own R0 columns (the
+//     TS-form A operands) and dS also into shared memory (for dQ)
+//   phase 2 (three interleaved MMA chains):
+//     dV  += P^T dOut       (A from TMEM)
+//     dK  += dS^T Q         (A from TMEM)
+//     dQ_s = dS K           -> TMEM R1        (A = dS from shared memory)
+//   the softmax warps then add dQ_s (fp32) into the global dQ accumulator
+//   with vector reductions; after the item, dK * scale and dV are stored.
+// TMEM columns: R0 [0,128), R1 [128,256), dV [256,256+D), dK [384,384+D).
+// Warp roles (320 threads): 0..7 the two groups, 8 TMA (K, V per item; Q,
+// dOut per step into a 2-slot ring, with lse and Dsum staged by its lanes),
+// 9 TMEM owner and MMA issuer.  Every mbarrier wait is bounded.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+
+#include "addr.cuh"
+#include "bsa_internal.h"
+#include "ptx_sm80.cuh"
+#include "sm100.cuh"
+#include "tc_common.h"
+#include "tc_device.cuh"
+
+namespace bsa {
+namespace {
+
+using namespace sm100;
+
+constexpr int kBThreads = 320;
+constexpr int kBLoadWarp = 8;
+constexpr int kBMmaWarp = 9;
+
+enum : int {
+  kBarKV = 0,       // K, V of the item landed
+  kBarKVEmpty = 1,  // the item's MMAs are done with K, V
+  kBarQD = 2,       // + slot: Q, dOut, lse, Dsum of a step landed
+  kBarQDEmpty = 4,  // + slot
+  kBarS = 6,        // S^T, dP^T of the step are in TMEM
+  kBarDS = 7,       // P, dS written (256 arrivals)
+  kBarP2 = 8,       // the step's dV, dK, dQ MMAs are done
+  kBarR1Free = 9,   // dQ of the step read out of TMEM (256 arrivals)
+  kBarAcc = 10,     // the item's dK, dV are final
+  kBarAccFree = 11, // dK, dV read out (256 arrivals)
+  kBarDrain = 12,
+  kNumBars = 13
+};
+
+template <int D>
+struct BLayout {
+  static constexpr int kBox = 128 * 128;
+  static constexpr int kTile = (D / 64) * kBox;
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + kTile;
+  static constexpr int kQ = kV + kTile;       // [2 slots]
+  static constexpr int kDO = kQ + 2 * kTile;  // [2 slots]
+  static constexpr int kDS = kDO + 2 * kTile; // dS: 128 kv rows x 128 q (two 64-q regions)
+  static constexpr int kStat = kDS + 2 * kBox;  // [2 slots][lse2 128 | Dsum 128] floats
+  static constexpr int kBars = kStat + 2 * 256 * 4;
+  static constexpr int kTmemPtr = kBars + kNumBars * 8;
+  static constexpr int kAbort = kTmemPtr + 4;
+  static constexpr int kBytes = kAbort + 4;
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+struct BItem {
+  int b, h2, u0, kvlen, wb, pg, gk, steps_ok;
+  BatchInfo bi;
+};
+
+__device__ __forceinline__ BItem b_item(const Problem &p, int id, int TK) {
+  BItem v;
+  const int ks = id % p.ksl;
+  v.gk = (id / p.ksl) % TK;
+  v.h2 = id / (p.ksl * TK);
+  v.b = p.kb_batch[v.gk];
+  v.bi = p.batch[v.b];
+  const int j = v.gk - v.bi.koff;
+  v.u0 = j * p.BKV + ks * 128;
+  v.kvlen = v.bi.kvlen;
+  v.wb = min(128, v.bi.kvst - v.u0);
+  v.pg = p.kv_layout == BSA_LAYOUT_PA_BBND ? kv_page(p, v.b, v.u0) : 0;
+  v.steps_ok = v.pg >= 0;
+  return v;
+}
+
+struct BStep {
+  int hh, e, st;  // q head within the group, inverted-list entry, 128-row step
+};
+
+__device__ __forceinline__ int64_t b_list(const Problem &p, const BItem &v, int hh, int TK) {
+  const int h1 = v.h2 * p.g + hh;
+  const int hi = p.Hidx == p.N1 ? h1 : v.h2;
+  return int64_t(hi) * TK + v.gk;
+}
+
+__device__ __forceinline__ BStep b_settle(const Problem &p, const BItem &v, BStep c, int TK) {
+  while (c.hh < p.g) {
+    const int64_t li = b_list(p, v, c.hh, TK);
+    const int len = p.inv_off[li + 1] - p.inv_off[li];
+    if (c.e < len) {
+      const int i = p.inv_list[p.inv_off[li] + c.e];
+      if (c.st < p.nsub && i * p.BQ + c.st * 128 < v.bi.qlen) return c;
+      ++c.e;
+      c.st = 0;
+      continue;
+    }
+    ++c.hh;
+    c.e = 0;
+    c.st = 0;
+  }
+  return c;
+}
+
+__device__ __forceinline__ BStep b_next(const Problem &p, const BItem &v, BStep c, int TK) {
+  ++c.st;
+  return b_settle(p, v, c, TK);
+}
+
+__device__ __forceinline__ int b_t0(const Problem &p, const BItem &v, const BStep &c, int TK) {
+  return p.inv_list[p.inv_off[b_list(p, v, c.hh, TK)] + c.e] * p.BQ + c.st * 128;
+}
+
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b),
+               "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(kBThreads, 1)
+    k_bwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
+             const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+             const __grid_constant__ CUtensorMap map_do) {
+  using L = BLayout<D>;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  extern __shared__ unsigned char smem_raw[];
+  const uint32_t base = smem_u32(smem_raw);
+  unsigned char *sbase = smem_raw;
+  if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(p.status + kStFlags, BSA_FLAG_INTERNAL);
+    return;
+  }
+  const uint32_t sK = base + L::kK, sV = base + L::kV, sQ = base + L::kQ, sDO = base + L::kDO;
+  const uint32_t sDS = base + L::kDS;
+  float *stat = reinterpret_cast<float *>(sbase + L::kStat);
+  auto bar = [&](int i) { return base + L::kBars + 8u * uint32_t(i); };
+  volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + L::kTmemPtr);
+  volatile int *abort = reinterpret_cast<volatile int *>(sbase + L::kAbort);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_items = int(p.status[kStBwdItems]);
+  const int TK = int(p.status[kStTK]);
+
+  if (tid == 0) {
+    mbar_init(bar(kBarKV), 1);
+    mbar_init(bar(kBarKVEmpty), 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar(kBarQD + s), 1);
+      mbar_init(bar(kBarQDEmpty + s), 1);
+    }
+    mbar_init(bar(kBarS), 1);
+    mbar_init(bar(kBarDS), 256);
+    mbar_init(bar(kBarP2), 1);
+    mbar_init(bar(kBarR1Free), 256);
+    mbar_init(bar(kBarAcc), 1);
+    mbar_init(bar(kBarAccFree), 256);
+    mbar_init(bar(kBarDrain), 1);
+    *abort = 0;
+    fence_barrier_init();
+  }
+  if (warp == kBMmaWarp) {
+    tmem_alloc(base + L::kTmemPtr, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tR0 = tmem, tR1 = tmem + 128u, tdV = tmem + 256u, tdK = tmem + 384u;
+  const float kLog2e = 1.4426950408889634f;
+
+  if (warp == kBLoadWarp) {
+    // ------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_v);
+      tma_prefetch_desc(&map_do);
+    }
+    uint32_t kv_it = 0, sk = 0;
+    int armed_kv = -1, armed_qd[2] = {-1, -1};
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const BItem v = b_item(p, p.bwd_items[it], TK);
+      if (!v.steps_ok) continue;
+      if (!(ok = wait_warp(bar(kBarKVEmpty), (kv_it & 1u) ^ 1u, abort, p.status))) break;
+      if (lane == 0) {
+        mbar_expect_tx(bar(kBarKV), 2 * L::kTile);
+        armed_kv = int(kv_it & 1u);
+        int c1, c2, c3;
+        if (p.kv_layout == BSA_LAYOUT_PA_BBND) { c1 = v.h2; c2 = v.u0 % p.page_size; c3 = v.pg; }
+        else if (p.kv_layout == BSA_LAYOUT_TND) { c1 = int(v.bi.kv_tok0) + v.u0; c2 = v.h2; c3 = 0; }
+        else { c1 = v.u0; c2 = v.h2; c3 = v.b; }
+        for (int h = 0; h < D / 64; ++h) {
+          tma_load_4d(sK + h * L::kBox, &map_k, bar(kBarKV), h * 64, c1, c2, c3);
+          tma_load_4d(sV + h * L::kBox, &map_v, bar(kBarKV), h * 64, c1, c2, c3);
+        }
+      }
+      ++kv_it;
+      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
+        const int slot = int(sk & 1u);
+        if (!(ok = wait_warp(bar(kBarQDEmpty + slot), ((sk >> 1) & 1u) ^ 1u, abort, p.status))) break;
+        const int h1 = v.h2 * p.g + c.hh;
+        const int t0 = b_t0(p, v, c, TK);
+        // lse (log2 units) and Dsum of the step's 128 query rows; rows past
+        // qlen get lse = +inf (so P = 0) and Dsum = 0
+        float *st = stat + slot * 256;
+        for (int j = lane; j < 128; j += 32) {
+          const int t = t0 + j;
+          float l2 = INFINITY, ds = 0.f;
+          if (t < v.bi.qlen) {
+            l2 = p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, h1, t)] * kLog2e;
+            if (!(l2 > -INFINITY)) l2 = INFINITY;  // a row with no selected key
+            const int64_t srow = p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq + t : v.bi.q_tok0 + t;
+            ds = p.dsum[srow * p.N1 + h1];
+          }
+          st[j] = l2;
+          st[128 + j] = ds;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          mbar_expect_tx(bar(kBarQD + slot), 2 * L::kTile);
+          armed_qd[slot] = int((sk >> 1) & 1u);
+          const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
+          const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
+          for (int h = 0; h < D / 64; ++h) {
+            tma_load_4d(sQ + slot * L::kTile + h * L::kBox, &map_q, bar(kBarQD + slot), h * 64, tok, h1, bb);
+            tma_load_4d(sDO + slot * L::kTile + h * L::kBox, &map_do, bar(kBarQD + slot), h * 64, tok, h1, bb);
+          }
+        }
+        __syncwarp();
+        ++sk;
+      }
+    }
+    if (*abort && lane == 0) {  // let every copy already issued land before the CTA exits
+      if (armed_kv >= 0) drain_wait(bar(kBarKV), uint32_t(armed_kv));
+      for (int s = 0; s < 2; ++s)
+        if (armed_qd[s] >= 0) drain_wait(bar(kBarQD + s), uint32_t(armed_qd[s]));
+    }
+  } else if (warp == kBMmaWarp) {
+    // ------------------------------------------------------- MMA issuer
+    constexpr uint32_t idSP = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
+    constexpr uint32_t idKV = idesc_f16(BF16, 128, D, false, true);     // dV, dK
+    constexpr uint32_t idQ = idesc_f16(BF16, 128, D, true, true);       // dQ
+    const uint64_t dKk = sw128_desc(sK, 16, 1024), dVk = sw128_desc(sV, 16, 1024);
+    const uint64_t dKmn = sw128_desc(sK, L::kBox, 1024);
+    const uint64_t dDS = sw128_desc(sDS, L::kBox, 1024);
+    auto kstep = [](int kk) { return uint64_t((kk >> 2) * (L::kBox >> 4) + (kk & 3) * 2); };
+    uint32_t kv_it = 0, sk = 0, item_n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const BItem v = b_item(p, p.bwd_items[it], TK);
+      if (!v.steps_ok) continue;
+      // the previous item's dK, dV must have been read out
+      if (item_n > 0 && !(ok = wait_warp(bar(kBarAccFree), (item_n - 1) & 1u, abort, p.status))) break;
+      ++item_n;
+      if (!(ok = wait_warp(bar(kBarKV), kv_it & 1u, abort, p.status))) break;
+      ++kv_it;
+      const int valid = v.kvlen - v.u0;
+      if (p.kv_layout == BSA_LAYOUT_PA_BBND && valid < 128) {
+        // rows of the last page past the used length may hold anything
+        // (even NaN): zero them in K and V so that they contribute nothing
+        for (int w = lane; w < (128 - valid) * 8 * (D / 64); w += 32) {
+          const int h = w / ((128 - valid) * 8), x = w % ((128 - valid) * 8);
+          reinterpret_cast<uint4 *>(sbase + L::kK + h * L::kBox)[valid * 8 + x] = make_uint4(0, 0, 0, 0);
+          reinterpret_cast<uint4 *>(sbase + L::kV + h * L::kBox)[valid * 8 + x] = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      bool first = true;
+      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
+        const int slot = int(sk & 1u);
+        if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
+        // R1 still holds the previous step's dQ until it has been read out
+        if (sk > 0 && !(ok = wait_warp(bar(kBarR1Free), (sk - 1) & 1u, abort, p.status))) break;
+        tc_fence_after();
+        const uint64_t dQk = sw128_desc(sQ + slot * L::kTile, 16, 1024);
+        const uint64_t dOk = sw128_desc(sDO + slot * L::kTile, 16, 1024);
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            mma_ss(tR0, dKk + kstep(kk), dQk + kstep(kk), idSP, kk > 0 ? 1u : 0u);
+            mma_ss(tR1, dVk + kstep(kk), dOk + kstep(kk), idSP, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(kBarS));
+        }
+        __syncwarp();
+        if (!(ok = wait_warp(bar(kBarDS), sk & 1u, abort, p.status))) break;
+        tc_fence_after();
+        const uint64_t dQmn = sw128_desc(sQ + slot * L::kTile, L::kBox, 1024);
+        const uint64_t dOmn = sw128_desc(sDO + slot * L::kTile, L::kBox, 1024);
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t pcol = uint32_t(64 * (kk >> 2) + 8 * (kk & 3));
+            const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+            mma_ts(tdV, tR0 + pcol, dOmn + uint64_t(kk * 128), idKV, acc);
+            mma_ts(tdK, tR0 + 32u + pcol, dQmn + uint64_t(kk * 128), idKV, acc);
+            mma_ss(tR1, dDS + uint64_t(kk * 128), dKmn + uint64_t(kk * 128), idQ, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar(kBarP2));
+          mma_commit(bar(kBarQDEmpty + slot));
+        }
+        __syncwarp();
+        first = false;
+        ++sk;
+      }
+      if (!ok) break;
+      if (lane == 0) {
+        mma_commit(bar(kBarKVEmpty));
+        mma_commit(bar(kBarAcc));
+      }
+      __syncwarp();
+    }
+    if (*abort && lane == 0) {  // let issued MMAs finish before TMEM is freed
+      mma_commit(bar(kBarDrain));
+      drain_wait(bar(kBarDrain), 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- the two softmax groups
+    const int wg = warp >> 2;
+    const int r = tid & 127;  // kv row (phase 1 / epilogue) or q row (dQ read-out)
+    const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
+    uint32_t sk = 0, item_n = 0;
+    bool ok = true;
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const BItem v = b_item(p, p.bwd_items[it], TK);
+      if (!v.steps_ok) {
+        if (tid == 0) atomicOr(p.status + kStFlags, BSA_FLAG_BAD_PAGE);
+        continue;
+      }
+      const bool kv_ok = v.u0 + r < v.kvlen;
+      int nsteps = 0;
+      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
+        const int slot = int(sk & 1u);
+        const int h1 = v.h2 * p.g + c.hh;
+        const int t0 = b_t0(p, v, c, TK);
+        if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
+        if (!(ok = wait_warp(bar(kBarS), sk & 1u, abort, p.status))) break;
+        tc_fence_after();
+        const float *lse2 = stat + slot * 256;
+        const float *dsum = lse2 + 128;
+        uint32_t pp[32], dd[32];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t xs[32], xd[32];
+          const uint32_t col = uint32_t(64 * wg + 32 * h);
+          tmem_ld32(tR0 + lane_off + col, xs);
+          tmem_ld32(tR1 + lane_off + col, xd);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c2 = 0; c2 < 32; c2 += 2) {
+            const int q = int(col) + c2;
+            const float p0 = kv_ok ? ex2(fmaf(__uint_as_float(xs[c2]), p.scale_log2, -lse2[q])) : 0.f;
+            const float p1 = kv_ok ? ex2(fmaf(__uint_as_float(xs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
+            const float s0 = p0 * (__uint_as_float(xd[c2]) - dsum[q]);
+            const float s1 = p1 * (__uint_as_float(xd[c2 + 1]) - dsum[q + 1]);
+            pp[16 * h + (c2 >> 1)] = MmaOp<T>::pack(p0, p1);
+            dd[16 * h + (c2 >> 1)] = MmaOp<T>::pack(s0, s1);
+          }
+        }
+        // P and dS into this group's own R0 columns (no other group reads
+        // them as S), dS also into shared memory for the dQ product
+        tmem_st32(tR0 + lane_off + uint32_t(64 * wg), pp);
+        tmem_st32(tR0 + lane_off + uint32_t(64 * wg + 32), dd);
+        {
+          // dS^T row r, q columns [64w, 64w+64): one 128-byte swizzled row
+          uint4 *row = reinterpret_cast<uint4 *>(sbase + L::kDS + wg * L::kBox + r * 128);
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            row[c ^ (r & 7)] = make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
+        }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(kBarDS));
+        // dQ of the step (lanes = q rows): add into the fp32 accumulator
+        if (!(ok = wait_warp(bar(kBarP2), sk & 1u, abort, p.status))) break;
+        tc_fence_after();
+        {
+          const int t = t0 + r;
+          const bool q_ok = t < v.bi.qlen;
+          const int64_t srow = p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq + t : v.bi.q_tok0 + t;
+          float *dq = p.dq_acc + (srow * p.N1 + h1) * D + (D / 2) * wg;
+#pragma unroll
+          for (int h = 0; h < D / 64; ++h) {
+            uint32_t x[32];
+            tmem_ld32(tR1 + lane_off + uint32_t((D / 2) * wg + 32 * h), x);
+            tmem_wait_ld();
+            if (q_ok) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 4)
+                red_add_v4(dq + 32 * h + c, __uint_as_float(x[c]), __uint_as_float(x[c + 1]),
+                           __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar(kBarR1Free));
+        ++sk;
+        ++nsteps;
+      }
+      if (!ok) break;
+      // ---- epilogue: dK * scale and dV, group w writes columns [w*D/2, (w+1)*D/2)
+      if (!(ok = wait_warp(bar(kBarAcc), item_n & 1u, abort, p.status))) break;
+      tc_fence_after();
+      if (r < v.wb) {
+        T *dkr = static_cast<T *>(p.dk) + kv_row(p, p.dk_sb, p.dk_sh, p.dk_st, v.bi, v.b, v.h2, v.u0 + r, v.pg);
+        T *dvr = static_cast<T *>(p.dv) + kv_row(p, p.dv_sb, p.dv_sh, p.dv_st, v.bi, v.b, v.h2, v.u0 + r, v.pg);
+        if (nsteps == 0) {
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            reinterpret_cast<uint4 *>(dkr + (D / 2) * wg)[c] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4 *>(dvr + (D / 2) * wg)[c] = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+      if (nsteps > 0) {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          const uint32_t col = uint32_t((D / 2) * wg + 32 * h);
+          uint32_t xk[32], xv[32];
+          tmem_ld32(tdK + lane_off + col, xk);
+          tmem_ld32(tdV + lane_off + col, xv);
+          tmem_wait_ld();
+          if (r < v.wb) {
+            T *dkr = static_cast<T *>(p.dk) + kv_row(p, p.dk_sb, p.dk_sh, p.dk_st, v.bi, v.b, v.h2, v.u0 + r, v.pg) + col;
+            T *dvr = static_cast<T *>(p.dv) + kv_row(p, p.dv_sb, p.dv_sh, p.dv_st, v.bi, v.b, v.h2, v.u0 + r, v.pg) + col;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint4 wk, wv;
+              wk.x = MmaOp<T>::pack(__uint_as_float(xk[c]) * p.scale, __uint_as_float(xk[c + 1]) * p.scale);
+              wk.y = MmaOp<T>::pack(__uint_as_float(xk[c + 2]) * p.scale, __uint_as_float(xk[c + 3]) * p.scale);
+              wk.z = MmaOp<T>::pack(__uint_as_float(xk[c + 4]) * p.scale, __uint_as_float(xk[c + 5]) * p.scale);
+              wk.w = MmaOp<T>::pack(__uint_as_float(xk[c + 6]) * p.scale, __uint_as_float(xk[c + 7]) * p.scale);
+              wv.x = MmaOp<T>::pack(__uint_as_float(xv[c]), __uint_as_float(xv[c + 1]));
+              wv.y = MmaOp<T>::pack(__uint_as_float(xv[c + 2]), __uint_as_float(xv[c + 3]));
+              wv.z = MmaOp<T>::pack(__uint_as_float(xv[c + 4]), __uint_as_float(xv[c + 5]));
+              wv.w = MmaOp<T>::pack(__uint_as_float(xv[c + 6]), __uint_as_float(xv[c + 7]));
+              *reinterpret_cast<uint4 *>(dkr + c) = wk;
+              *reinterpret_cast<uint4 *>(dvr + c) = wv;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(kBarAccFree));
+      ++item_n;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D, bool BF16>
+cudaError_t launch_bwd_tc(const Problem &p, const BwdMaps &m, cudaStream_t s) {
+  const int smem = BLayout<D>::kBytes > 120 * 1024 ? BLayout<D>::kBytes : 120 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = p.bwd_slots < num_sms() ? p.bwd_slots : num_sms();
+  if (grid <= 0) return cudaSuccess;
+  k_bwd_tc<D, BF16><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_bwd_main(const Problem &p, cudaStream_t s) {
+  BwdMaps m;
+  cudaError_t e = make_bwd_maps(p, m);
+  if (e != cudaSuccess) return e;
+  if (p.dtype == BSA_BF16)
+    return p.D == 64 ? launch_bwd_tc<64, true>(p, m, s) : launch_bwd_tc<128, true>(p, m, s);
+  return p.D == 64 ? launch_bwd_tc<64, false>(p, m, s) : launch_bwd_tc<128, false>(p, m, s);
+}
+
+}  // namespace bsa

@@ -5,25 +5,31 @@
 // row over the kv tokens of the blocks in the row's compacted index row,
 // lse = natural log of the sum of exp(scale * q.k).
 //
-// One persistent CTA per SM; each work item is 128 query rows of one head.
-// Warp roles (256 threads):
-//   warp 0      TMA producer: Q tile once per item, then K and V 128-row
-//               chunks of the selected kv blocks into a 2-stage ring.
-//   warp 1      TMEM owner and MMA issuer (one elected lane):
-//                 S_j = Q K_j^T        (SS form, fp32 accumulator in TMEM)
-//                 O  += P_j V_j        (TS form, P read from TMEM)
-//   warps 4..7  softmax warpgroup, one query row per thread (TMEM lane):
-//               reads S_j, masks kv columns past kvlen, keeps the running
-//               max m (log2 domain) and sum l, writes P_j = exp2(s - m)
-//               as packed 16-bit pairs back over S_j, and rescales O only
-//               when the running max grew by more than 2^8 (so P stays
-//               below 256); epilogue O / l and lse = (m + log2 l) ln 2.
-// S is double-buffered in TMEM so S_{j+1} = Q K_{j+1}^T runs on the tensor
-// cores while the softmax warpgroup works on S_j.
-// TMEM columns: [0,128) S buffer 0, [128,256) S buffer 1, [256,256+D) O.
-// Every wait on an mbarrier is bounded; on expiry the CTA raises
+// One persistent CTA per SM; each work item is 128 query rows of one head,
+// walked over 128-row kv chunks t of the selected blocks.
+// Warp roles (352 threads):
+//   warp 8      TMA: the Q tile once per item, then K chunks (3-stage ring)
+//   warp 10     TMA: the matching V chunks (3-stage ring)
+//   warp 9      TMEM owner and MMA issuer (one elected lane).  It keeps two
+//               independent accumulation chains in flight: the P_t V_t
+//               product (TS form, P read from TMEM) is interleaved MMA by MMA
+//               with S_{t+2} = Q K_{t+2}^T (SS form), since one chain of
+//               dependent MMAs into a single accumulator runs at about half
+//               the tensor rate.  Descriptors are precomputed and advanced
+//               by adding to their address field.
+//   warps 0..7  two softmax warpgroups; thread (group w, row r) owns kv
+//               columns [64w, 64w+64) of query row r in every chunk.  The
+//               running max m (log2 domain) is kept stale until a row's max
+//               grows by more than 2^8 (P stays below 256); only then are the
+//               two halves' maxima exchanged, O and the partial sums l
+//               rescaled.  P = exp2(s*scale*log2 e - m) overwrites S as
+//               16-bit pairs.  Epilogue: out = O / (l_0 + l_1),
+//               lse = (m + log2(l_0 + l_1)) ln 2.
+// TMEM columns: three S/P buffers [0,128), [128,256), [256,384); O [384,384+D).
+// Every mbarrier wait is bounded (2 s); on expiry the CTA raises
 // BSA_FLAG_TIMEOUT, drains its in-flight copies and MMAs, frees TMEM and
-// returns.
+// returns.  The two softmax warpgroups meet only on mbarriers, so an abort
+// never strands one of them on a hardware barrier.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -34,45 +40,56 @@
 #include "ptx_sm80.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
+#include "tc_device.cuh"
 
 namespace bsa {
 namespace {
 
 using namespace sm100;
 
-constexpr int kTcThreads = 384;
-constexpr int kStages = 2;
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s: any legitimate wait is far shorter
-constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O when m grows by > 2^8
+constexpr int kSoftmaxGroups = 2;  // warpgroups sharing the kv columns of a chunk
+constexpr int kSoftmaxThreads = 128 * kSoftmaxGroups;
+constexpr int kTcThreads = kSoftmaxThreads + 96;  // + Q/K loads, MMA, V loads
+constexpr int kStages = 3;       // depth of the K ring and of the V ring
+constexpr int kSBufs = 3;        // S / P buffers in TMEM
+constexpr int kLoadWarp = 4 * kSoftmaxGroups;
+constexpr int kMmaWarp = kLoadWarp + 1;
+constexpr int kVLoadWarp = kLoadWarp + 2;
+constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
+constexpr float kRescaleThreshold = 8.0f;    // log2 units
 
 // barrier slots
 enum : int {
   kBarQFull = 0,
   kBarQEmpty = 1,
-  kBarKFull = 2,   // + stage
-  kBarKEmpty = 4,  // + stage
-  kBarVFull = 6,   // + stage
-  kBarVEmpty = 8,  // + stage
-  kBarSFull = 10,  // + buffer
-  kBarPFull = 12,  // + buffer
-  kBarPVDone = 14,  // + (chunk index % 2): P_t V_t is in O
-  kBarDrain = 16,
-  kNumBars = 17
+  kBarKFull = 2,    // + K stage
+  kBarKEmpty = 5,   // + K stage
+  kBarVFull = 8,    // + V stage
+  kBarVEmpty = 11,  // + V stage
+  kBarSFull = 14,   // + S buffer
+  kBarPFull = 17,   // + S buffer (one arrival per softmax thread)
+  kBarPVDone = 20,  // + (chunk index & 1): P_t V_t is in O
+  kBarXchg = 22,    // the softmax groups' rendezvous (one arrival per softmax thread)
+  kBarDrain = 23,
+  kNumBars = 24
 };
 
 template <int D>
 struct Layout {
-  static constexpr int kBox = 128 * 128;              // one 128-row x 64-col 16-bit box
-  static constexpr int kTile = (D / 64) * kBox;       // Q / K / V tile
+  static constexpr int kBox = 128 * 128;         // one 128-row x 64-col 16-bit box
+  static constexpr int kTile = (D / 64) * kBox;  // Q / K / V tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBars = kV + kStages * kTile;
-  static constexpr int kXchg = kBars + kNumBars * 8 + 8;  // [2][2][128] floats (max, sum)
-  static constexpr int kTmemPtr = kXchg + 2 * 2 * 128 * 4;
+  static constexpr int kFlags = kBars + kNumBars * 8;                 // [2][softmax warps] u32
+  static constexpr int kXsum = kFlags + 2 * 4 * kSoftmaxGroups * 4;   // [groups][128] sums
+  static constexpr int kTmemPtr = kXsum + kSoftmaxGroups * 128 * 4;
   static constexpr int kAbort = kTmemPtr + 4;
   static constexpr int kBytes = kAbort + 4;
-  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+  // the dynamic shared window starts 1024-byte aligned (checked at run time)
+  static constexpr int kAlloc = kBytes;
+  static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
 struct Chunk {
@@ -133,49 +150,6 @@ __device__ __forceinline__ ItemView item_view(const Problem &p, int id) {
   return v;
 }
 
-__device__ __forceinline__ uint64_t global_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-// Bounded wait: gives up after kWaitNs of wall time (raising the abort flag
-// and BSA_FLAG_TIMEOUT), or as soon as another role has aborted.
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort,
-                                         uint32_t *status) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*abort) return false;
-      if (global_ns() - t0 > kWaitNs) {
-        *abort = 1;
-        atomicOr(status + kStFlags, BSA_FLAG_TIMEOUT);
-        return false;
-      }
-    }
-  }
-}
-
-// the same, agreed by the whole warp (tcgen05 .sync.aligned ops follow)
-__device__ __forceinline__ bool wait_warp(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          uint32_t *status) {
-  const bool r = wait_bar(bar, parity, abort, status);
-  return __all_sync(0xffffffffu, r);
-}
-
-__device__ __forceinline__ void named_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(threads) : "memory");
-}
-
-// drain wait on the abort path: bounded, result ignored
-__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
-  const uint64_t t0 = global_ns();
-  while (!mbar_try_wait(bar, parity) && global_ns() - t0 < kWaitNs) {
-  }
-}
-
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_fwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
@@ -183,9 +157,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using L = Layout<D>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ unsigned char smem_raw[];
-  const uint32_t raw_base = smem_u32(smem_raw);
-  const uint32_t base = (raw_base + 1023u) & ~1023u;
-  unsigned char *sbase = smem_raw + (base - raw_base);
+  const uint32_t base = smem_u32(smem_raw);
+  unsigned char *sbase = smem_raw;
+  if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
+    if (threadIdx.x == 0) atomicOr(p.status + kStFlags, BSA_FLAG_INTERNAL);
+    return;
+  }
   const uint32_t sQ = base + L::kQ, sK = base + L::kK, sV = base + L::kV;
   auto bar = [&](int i) { return base + L::kBars + 8u * uint32_t(i); };
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + L::kTmemPtr);
@@ -202,16 +179,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(bar(kBarKEmpty + s), 1);
       mbar_init(bar(kBarVFull + s), 1);
       mbar_init(bar(kBarVEmpty + s), 1);
-      mbar_init(bar(kBarSFull + s), 1);
-      mbar_init(bar(kBarPFull + s), 128);
+    }
+    for (int b = 0; b < kSBufs; ++b) {
+      mbar_init(bar(kBarSFull + b), 1);
+      mbar_init(bar(kBarPFull + b), kSoftmaxThreads);
     }
     mbar_init(bar(kBarPVDone), 1);
     mbar_init(bar(kBarPVDone + 1), 1);
+    mbar_init(bar(kBarXchg), kSoftmaxThreads);
     mbar_init(bar(kBarDrain), 1);
     *abort = 0;
     fence_barrier_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(base + L::kTmemPtr, 512);
     tmem_relinquish();
   }
@@ -219,31 +199,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS0 = tmem, tO0 = tmem + 256;  // S_w at tS0 + 128w, O_w at tO0 + D*w
+  const uint32_t tS0 = tmem, tO = tmem + uint32_t(kSBufs) * 128u;
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == kLoadWarp || warp == kVLoadWarp) {
+    // ----------------------------------------------------- TMA producers
+    const bool is_k = warp == kLoadWarp;
     if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_k);
-      tma_prefetch_desc(&map_v);
+      const CUtensorMap *map = is_k ? &map_k : &map_v;
+      if (is_k) tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(map);
+      const uint32_t ring = is_k ? sK : sV;
+      const int full0 = is_k ? kBarKFull : kBarVFull, empty0 = is_k ? kBarKEmpty : kBarVEmpty;
       uint32_t kv_it = 0, q_it = 0;
-      int armed_q = -1, armed_k[kStages] = {-1, -1}, armed_v[kStages] = {-1, -1};
+      int armed_q = -1, armed[kStages] = {-1, -1, -1};
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const ItemView v = item_view(p, p.fwd_items[it]);
         if (count_chunks(p, v) == 0) continue;
-        ok = wait_bar(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status);
-        if (!ok) break;
-        mbar_expect_tx(bar(kBarQFull), L::kTile);
-        armed_q = int(q_it & 1u);
-        {
+        if (is_k) {
+          if (!(ok = wait_bar(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status))) break;
+          mbar_expect_tx(bar(kBarQFull), L::kTile);
+          armed_q = int(q_it & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + v.t0 : v.t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
           for (int h = 0; h < D / 64; ++h)
             tma_load_4d(sQ + h * L::kBox, &map_q, bar(kBarQFull), h * 64, tok, v.h1, bb);
+          ++q_it;
         }
-        ++q_it;
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) {
           const int s = int(kv_it % kStages);
           const uint32_t ph = (kv_it / kStages) & 1u;
@@ -254,61 +236,76 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (p.kv_layout == BSA_LAYOUT_PA_BBND) { c1 = v.h2; c2 = u0 % p.page_size; c3 = pg; }
           else if (p.kv_layout == BSA_LAYOUT_TND) { c1 = int(v.bi.kv_tok0) + u0; c2 = v.h2; c3 = 0; }
           else { c1 = u0; c2 = v.h2; c3 = v.b; }
-          if (!(ok = wait_bar(bar(kBarKEmpty + s), ph ^ 1u, abort, p.status))) break;
-          mbar_expect_tx(bar(kBarKFull + s), L::kTile);
-          armed_k[s] = int(ph);
+          if (!(ok = wait_bar(bar(empty0 + s), ph ^ 1u, abort, p.status))) break;
+          mbar_expect_tx(bar(full0 + s), L::kTile);
+          armed[s] = int(ph);
           for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sK + s * L::kTile + h * L::kBox, &map_k, bar(kBarKFull + s), h * 64, c1, c2, c3);
-          if (!(ok = wait_bar(bar(kBarVEmpty + s), ph ^ 1u, abort, p.status))) break;
-          mbar_expect_tx(bar(kBarVFull + s), L::kTile);
-          armed_v[s] = int(ph);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sV + s * L::kTile + h * L::kBox, &map_v, bar(kBarVFull + s), h * 64, c1, c2, c3);
+            tma_load_4d(ring + s * L::kTile + h * L::kBox, map, bar(full0 + s), h * 64, c1, c2, c3);
           ++kv_it;
         }
       }
       if (*abort) {  // let every copy already issued land before the CTA exits
         if (armed_q >= 0) drain_wait(bar(kBarQFull), uint32_t(armed_q));
-        for (int s = 0; s < kStages; ++s) {
-          if (armed_k[s] >= 0) drain_wait(bar(kBarKFull + s), uint32_t(armed_k[s]));
-          if (armed_v[s] >= 0) drain_wait(bar(kBarVFull + s), uint32_t(armed_v[s]));
-        }
+        for (int s = 0; s < kStages; ++s)
+          if (armed[s] >= 0) drain_wait(bar(full0 + s), uint32_t(armed[s]));
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     constexpr uint32_t idS = idesc_f16(BF16, 128, 128, false, false);
     constexpr uint32_t idPV = idesc_f16(BF16, 128, D, false, true);
+    // descriptors: K-major Q / K (a 16-element K step is +32 B, the second
+    // 64-column box +16 KB); MN-major V (a 16-row K step is +2 KB, the two
+    // 64-column halves 16 KB apart)
+    const uint64_t dQ = sw128_desc(sQ, 16, 1024);
+    const uint64_t dK = sw128_desc(sK, 16, 1024);
+    const uint64_t dV = sw128_desc(sV, L::kBox, 1024);
+    auto kstep = [](int kk) { return uint64_t((kk >> 2) * (L::kBox >> 4) + (kk & 3) * 2); };
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
-    auto issue_pv = [&](uint32_t t, bool first, int valid) {
-      const int s = int(t % kStages);
-      const uint32_t ph = (t / kStages) & 1u;
-      if (!(ok = wait_warp(bar(kBarPFull + s), ph, abort, p.status))) return;
-      if (!(ok = wait_warp(bar(kBarVFull + s), ph, abort, p.status))) return;
-      if (p.kv_layout == BSA_LAYOUT_PA_BBND && valid < 128) {
-        // rows of the last page past the used length may hold anything
-        // (even NaN); their P is 0, so make their V exactly 0 as well
-        uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + s * L::kTile);
-        const int per_half = (128 - valid) * 8;  // 16-byte words per 64-column half
-        for (int w = lane; w < per_half * (D / 64); w += 32) {
-          const int h = w / per_half, x = w % per_half;
-          vt[h * (L::kBox / 16) + valid * 8 + x] = make_uint4(0, 0, 0, 0);
+    // Issue P_pv V_pv (pv >= 0) interleaved with S_sa, S_sb (>= 0), then
+    // signal: S_full / K_empty per S, PV_done / V_empty for the product,
+    // Q_empty after the item's last S (last_s).
+    auto issue = [&](int64_t pv, bool pv_first, int pv_valid, int64_t sa, int64_t sb,
+                     int64_t last_s) {
+      if (pv >= 0) {
+        if (!(ok = wait_warp(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
+        if (!(ok = wait_warp(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
+        if (p.kv_layout == BSA_LAYOUT_PA_BBND && pv_valid < 128) {
+          // rows of the last page past the used length may hold anything
+          // (even NaN); their P is 0, so make their V exactly 0 as well
+          uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + int(pv % kStages) * L::kTile);
+          const int per_half = (128 - pv_valid) * 8;  // 16-byte words per 64-column half
+          for (int w = lane; w < per_half * (D / 64); w += 32) {
+            const int h = w / per_half, x = w % per_half;
+            vt[h * (L::kBox / 16) + pv_valid * 8 + x] = make_uint4(0, 0, 0, 0);
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
         }
-        fence_proxy_async_smem();
-        __syncwarp();
       }
+      if (sa >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
+      if (sb >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t a_tmem = tS0 + uint32_t(s) * 128u;
+        const uint32_t pa = tS0 + uint32_t(pv % kSBufs) * 128u;
+        const uint64_t vd = dV + uint64_t((pv % kStages) * (L::kTile >> 4));
+        const uint32_t da = tS0 + uint32_t(sa % kSBufs) * 128u, db = tS0 + uint32_t(sb % kSBufs) * 128u;
+        const uint64_t ka = dK + uint64_t((sa % kStages) * (L::kTile >> 4));
+        const uint64_t kb = dK + uint64_t((sb % kStages) * (L::kTile >> 4));
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bdesc = sw128_desc(sV + s * L::kTile + kk * 2048, L::kBox, 1024);
-          mma_ts(tO0 + uint32_t(s) * D, a_tmem + uint32_t(kk) * 8u, bdesc, idPV,
-                 (first && kk == 0) ? 0u : 1u);
+          if (pv >= 0)
+            mma_ts(tO, pa + uint32_t(kk) * 8u, vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
+          if (kk < D / 16) {
+            if (sa >= 0) mma_ss(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+            if (sb >= 0) mma_ss(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          }
         }
-        mma_commit(bar(kBarPVDone + s));
-        mma_commit(bar(kBarVEmpty + s));
+        if (sa >= 0) { mma_commit(bar(kBarSFull + int(sa % kSBufs))); mma_commit(bar(kBarKEmpty + int(sa % kStages))); }
+        if (sb >= 0) { mma_commit(bar(kBarSFull + int(sb % kSBufs))); mma_commit(bar(kBarKEmpty + int(sb % kStages))); }
+        if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit(bar(kBarQEmpty));
+        if (pv >= 0) { mma_commit(bar(kBarPVDone + int(pv & 1))); mma_commit(bar(kBarVEmpty + int(pv % kStages))); }
       }
       __syncwarp();
     };
@@ -318,131 +315,144 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (n == 0) continue;
       if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
       ++q_it;
-      int prev_valid = 128;
+      const int64_t t0 = kv_it, last = kv_it + n - 1;
+      issue(-1, false, 128, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
       Chunk ch = settle(p, v, Chunk{0, 0});
       for (int j = 0; j < n && ok; ++j) {
-        const int s = int(kv_it % kStages);
-        const uint32_t ph = (kv_it / kStages) & 1u;
-        if (!(ok = wait_warp(bar(kBarKFull + s), ph, abort, p.status))) break;
-        tc_fence_after();
-        if (lane == 0) {
-          const uint32_t d_tmem = tS0 + uint32_t(s) * 128u;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = uint32_t(kk >> 2) * L::kBox + uint32_t(kk & 3) * 32u;
-            mma_ss(d_tmem, sw128_desc(sQ + off, 16, 1024),
-                   sw128_desc(sK + s * L::kTile + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bar(kBarSFull + s));
-          mma_commit(bar(kBarKEmpty + s));
-          if (j == n - 1) mma_commit(bar(kBarQEmpty));
-        }
-        __syncwarp();
-        if (j >= 1) issue_pv(kv_it - 1, j <= 2, prev_valid);
-        prev_valid = v.kvlen - v.u0(ch);
+        const int valid = v.kvlen - v.u0(ch);
+        issue(t0 + j, j == 0, valid, j + 2 < n ? t0 + j + 2 : -1, -1, last);
         ch = next_chunk(p, v, ch);
-        ++kv_it;
       }
-      if (ok) issue_pv(kv_it - 1, n <= 2, prev_valid);
+      kv_it += uint32_t(n);
     }
     if (*abort && lane == 0) {  // let issued MMAs finish before TMEM is freed
       mma_commit(bar(kBarDrain));
       drain_wait(bar(kBarDrain), 0);
     }
     __syncwarp();
-  } else if (warp >= 4) {
-    // ------------------------------------------- two softmax warpgroups
-    // Warpgroup w takes the chunks whose global index t has t % 2 == w: its
-    // own S buffer, O accumulator, running max and sum (a split of the kv
-    // range inside the CTA); the halves are merged in the epilogue.
-    const int wg = (warp - 4) >> 2;
-    const int r = (tid - 128) & 127;                        // query row = TMEM lane
+  } else if (warp < kLoadWarp) {
+    // --------------------------------------------- softmax warpgroups
+    const int wg = warp >> 2;
+    const int r = tid & 127;  // query row = TMEM lane
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
-    const uint32_t tS = tS0 + uint32_t(wg) * 128u + lane_off;
-    const uint32_t tOw = tO0 + uint32_t(wg) * D + lane_off;
-    float *xm = reinterpret_cast<float *>(sbase + L::kXchg);  // [2][128] max
-    float *xl = xm + 256;                                     // [2][128] sum
+    volatile uint32_t *flags = reinterpret_cast<volatile uint32_t *>(sbase + L::kFlags);
+    float *xsum = reinterpret_cast<float *>(sbase + L::kXsum);
     const float kLn2 = 0.6931471805599453f;
-    uint32_t kv_it = 0, own = 0;  // global chunk counter; chunks this group took
+    constexpr int kWarps = 4 * kSoftmaxGroups;
+    uint32_t kv_it = 0, x_it = 0;  // global chunk counter; rendezvous counter
     bool ok = true;
+    // all softmax threads meet here (bounded: an aborted peer cannot strand us)
+    auto rendezvous = [&]() {
+      mbar_arrive(bar(kBarXchg));
+      ok = wait_warp(bar(kBarXchg), x_it & 1u, abort, p.status);
+      ++x_it;
+      return ok;
+    };
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const ItemView v = item_view(p, p.fwd_items[it]);
       float m = -INFINITY, l = 0.f;
       int n = 0;
-      for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
-           ch = next_chunk(p, v, ch), ++n, ++kv_it) {
-        if (int(kv_it & 1u) != wg) continue;
-        if (!(ok = wait_warp(bar(kBarSFull + wg), own & 1u, abort, p.status))) break;
-        tc_fence_after();
-        const int valid = v.kvlen - v.u0(ch);  // kv columns of this chunk that exist
-        // the whole 128-column row in one round trip
-        uint32_t x[4][32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + uint32_t(q) * 32u, x[q]);
-        tmem_wait_ld();
-        if (valid < 128) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (q * 32 + c >= valid) x[q][c] = __float_as_uint(-INFINITY);
+      {
+        // the chunk walk needs only the index row, its length, kvlen and the
+        // batch; the rest of the item is re-derived for the epilogue
+        ItemView v;
+        {
+          const ItemView full = item_view(p, p.fwd_items[it]);
+          v.crow = full.crow;
+          v.ncnt = full.ncnt;
+          v.kvlen = full.kvlen;
+          v.b = full.b;
+          v.ksl = p.ksl;
+          v.BKV = p.BKV;
         }
-        float pm[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) pm[k] = -INFINITY;
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int c = 0; c < 32; ++c) pm[c & 7] = fmaxf(pm[c & 7], __uint_as_float(x[q][c]));
-        const float cmax = fmaxf(fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])),
-                                 fmaxf(fmaxf(pm[4], pm[5]), fmaxf(pm[6], pm[7]))) * p.scale_log2;
-        // running max: adopted on the group's first chunk; afterwards kept
-        // stale until it falls more than 2^8 behind (then O and l rescale)
-        const bool first = m == -INFINITY;
-        const bool grow = __any_sync(0xffffffffu, !first && cmax > m + kRescaleThreshold);
-        const float m_new = first ? cmax : (grow ? fmaxf(m, cmax) : m);
-        const float alpha = (first || !grow) ? 1.f : ex2(m - m_new);
-        m = m_new;
-        // P = exp2(scale*log2(e)*s - m), written over S as 16-bit pairs
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int q = 0; q < 2; ++q)
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const float e0 = ex2(fmaf(__uint_as_float(x[2 * h + q][c]), p.scale_log2, -m));
-              const float e1 = ex2(fmaf(__uint_as_float(x[2 * h + q][c + 1]), p.scale_log2, -m));
-              ps[(c >> 1) & 3] += e0 + e1;
-              pk[q * 16 + (c >> 1)] = MmaOp<T>::pack(e0, e1);
-            }
-          tmem_st32(tS + uint32_t(h) * 32u, pk);
-        }
-        l = l * alpha + ((ps[0] + ps[1]) + (ps[2] + ps[3]));
-        if (grow) {
-          // O may only be rescaled once this group's previous P V (t - 2,
-          // same accumulator) has landed in it
-          const uint32_t t = kv_it - 2;
-          if (!(ok = wait_warp(bar(kBarPVDone + wg), (t / 2) & 1u, abort, p.status))) break;
+        for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
+             ch = next_chunk(p, v, ch), ++n, ++kv_it) {
+          const int b = int(kv_it % kSBufs);
+          if (!(ok = wait_warp(bar(kBarSFull + b), (kv_it / kSBufs) & 1u, abort, p.status))) break;
           tc_fence_after();
+          const uint32_t tS = tS0 + uint32_t(b) * 128u + lane_off;
+          const int valid_all = v.kvlen - v.u0(ch);       // kv columns of the chunk that exist
+          const int valid = valid_all - kCols * wg;        // of this group's columns
+          uint32_t x[kCols];
+          tmem_ld_cols<kCols>(tS + uint32_t(kCols * wg), x);
+          tmem_wait_ld();
+          if (valid < kCols) {
 #pragma unroll
-          for (int q = 0; q < D / 32; ++q) {
-            uint32_t o[32];
-            tmem_ld32(tOw + uint32_t(q) * 32u, o);
+            for (int c = 0; c < kCols; ++c)
+              if (c >= valid) x[c] = __float_as_uint(-INFINITY);
+          }
+          float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < kCols; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(x[c]));
+          const float hmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
+          // does any row of this warp's columns need a new max?
+          const bool first = m == -INFINITY;
+          const uint32_t need = __any_sync(0xffffffffu, first || hmax > m + kRescaleThreshold) ? 1u : 0u;
+          if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
+          // after this rendezvous every S column has been read: P may overwrite S
+          if (!rendezvous()) break;
+          // one decision for the whole CTA, so that every group takes the
+          // same number of rendezvous
+          uint32_t any = 0;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) any |= flags[(kv_it & 1u) * kWarps + w];
+          float alpha = 1.f;
+          const bool grow = any != 0u;
+          if (grow) {
+            // the full row max: the other groups' columns are still S in TMEM
+            float cm = hmax;
+#pragma unroll 1
+            for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) {
+              if (g2 == wg) continue;
+              uint32_t y[kCols];
+              tmem_ld_cols<kCols>(tS + uint32_t(kCols * g2), y);
+              tmem_wait_ld();
+              float ym = -INFINITY;
+              const int vy = valid_all - kCols * g2;
+#pragma unroll
+              for (int c = 0; c < kCols; ++c)
+                if (c < vy) ym = fmaxf(ym, __uint_as_float(y[c]));
+              cm = fmaxf(cm, ym * p.scale_log2);
+            }
+            // nobody overwrites S with P before every thread has read it
+            if (!rendezvous()) break;
+            const float m_new = fmaxf(m, cm);
+            alpha = first ? 1.f : ex2(m - m_new);
+            m = m_new;
+          }
+          // P = exp2(scale*log2(e)*s - m) over this group's columns
+          float ps[2] = {0.f, 0.f};
+          uint32_t pk[kCols / 2];
+#pragma unroll
+          for (int c = 0; c < kCols; c += 2) {
+            const float e0 = ex2(fmaf(__uint_as_float(x[c]), p.scale_log2, -m));
+            const float e1 = ex2(fmaf(__uint_as_float(x[c + 1]), p.scale_log2, -m));
+            ps[(c >> 1) & 1] += e0 + e1;
+            pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+          }
+          tmem_st_cols<kCols / 2>(tS + uint32_t((kCols / 2) * wg), pk);
+          l = l * alpha + (ps[0] + ps[1]);
+          if (grow && !first && __any_sync(0xffffffffu, alpha != 1.f)) {
+            // O may only be rescaled once P_{t-1} V_{t-1} (and so every
+            // earlier product, the tensor pipe being in order) has landed
+            const uint32_t t = kv_it - 1;
+            if (!(ok = wait_warp(bar(kBarPVDone + int(t & 1u)), (t / 2) & 1u, abort, p.status))) break;
+            tc_fence_after();
+            const uint32_t col = tO + lane_off + uint32_t(wg * (D / kSoftmaxGroups));
+            uint32_t o[D / kSoftmaxGroups];
+            tmem_ld_cols<D / kSoftmaxGroups>(col, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-            tmem_st32(tOw + uint32_t(q) * 32u, o);
+            for (int c = 0; c < D / kSoftmaxGroups; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+            tmem_st_cols<D / kSoftmaxGroups>(col, o);
           }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(kBarPFull + b));
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(kBarPFull + wg));
-        ++own;
       }
       if (!ok) break;
-      // ---- epilogue: merge the two groups' partial results
+      // ---- epilogue: out = O / sum of the groups' l; group w writes D/4 columns
+      const ItemView v = item_view(p, p.fwd_items[it]);
       const bool live = r < v.rows;
       T *orow = static_cast<T *>(p.out) + q_row(p.o_sb, p.o_sh, p.o_st, v.bi, v.b, v.h1, v.t0 + r);
       if (n > 0) {
@@ -450,48 +460,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!(ok = wait_warp(bar(kBarPVDone + int(t & 1u)), (t / 2) & 1u, abort, p.status))) break;
         tc_fence_after();
       }
-      xm[wg * 128 + r] = m;
-      xl[wg * 128 + r] = l;
-      named_sync(1, 256);
-      const float m0 = xm[r], m1 = xm[128 + r], l0 = xl[r], l1 = xl[128 + r];
-      const float M = fmaxf(m0, m1);
-      const float a0 = m0 == -INFINITY ? 0.f : ex2(m0 - M);
-      const float a1 = m1 == -INFINITY ? 0.f : ex2(m1 - M);
-      const float Lsum = l0 * a0 + l1 * a1;
-      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      // group w writes columns [w*D/2, (w+1)*D/2) from both accumulators
+      xsum[wg * 128 + r] = l;
+      if (!rendezvous()) break;
+      float Lsum = 0.f;
 #pragma unroll
-      for (int q = 0; q < D / 32; ++q) {
-        const uint32_t col = uint32_t(wg) * (D / 2) + uint32_t(q) * 16u;
-        uint32_t o0[16], o1[16];
-        tmem_ld16(tO0 + lane_off + col, o0);
-        tmem_ld16(tO0 + uint32_t(D) + lane_off + col, o1);
-        tmem_wait_ld();
-        if (live) {
-          uint4 w[2];
-          uint32_t *wp = reinterpret_cast<uint32_t *>(w);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const float y0 = (a0 > 0.f ? __uint_as_float(o0[2 * c]) * a0 : 0.f) +
-                             (a1 > 0.f ? __uint_as_float(o1[2 * c]) * a1 : 0.f);
-            const float y1 = (a0 > 0.f ? __uint_as_float(o0[2 * c + 1]) * a0 : 0.f) +
-                             (a1 > 0.f ? __uint_as_float(o1[2 * c + 1]) * a1 : 0.f);
-            wp[c] = MmaOp<T>::pack(y0 * inv, y1 * inv);
-          }
-          reinterpret_cast<uint4 *>(orow + col)[0] = w[0];
-          reinterpret_cast<uint4 *>(orow + col)[1] = w[1];
-        }
-      }
+      for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) Lsum += xsum[g2 * 128 + r];
       if (wg == 0 && live && p.lse)
         p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1, v.t0 + r)] =
-            Lsum > 0.f ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+            Lsum > 0.f ? (m + __log2f(Lsum)) * kLn2 : -INFINITY;
+      const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+      constexpr int kOc = D / kSoftmaxGroups;  // output columns per group
+      if (n > 0) {
+#pragma unroll
+        for (int q = 0; q < kOc / 16; ++q) {
+          const uint32_t col = uint32_t(wg * kOc + q * 16);
+          uint32_t o[16];
+          tmem_ld16(tO + lane_off + col, o);
+          tmem_wait_ld();
+          if (live) {
+            uint4 w[2];
+            uint32_t *wp = reinterpret_cast<uint32_t *>(w);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              wp[c] = MmaOp<T>::pack(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
+            reinterpret_cast<uint4 *>(orow + col)[0] = w[0];
+            reinterpret_cast<uint4 *>(orow + col)[1] = w[1];
+          }
+        }
+      } else if (live) {
+#pragma unroll
+        for (int c = 0; c < kOc / 8; ++c)
+          reinterpret_cast<uint4 *>(orow + wg * kOc)[c] = make_uint4(0, 0, 0, 0);
+      }
       tc_fence_before();
-      named_sync(1, 256);  // both groups are done with O and the exchange slots
+      // every group is done with O and the exchange slots before the next item
+      if (!rendezvous()) break;
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -150,6 +150,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[15])
       : "memory");
 }
+// N (a multiple of 16) consecutive columns into / out of r[0..N)
+template <int N>
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t *r) {
+  static_assert(N % 16 == 0, "16-column granularity");
+#pragma unroll
+  for (int c = 0; c + 32 <= N; c += 32)
+    tmem_ld32(taddr + uint32_t(c), *reinterpret_cast<uint32_t(*)[32]>(r + c));
+  if constexpr (N % 32 == 16)
+    tmem_ld16(taddr + uint32_t(N - 16), *reinterpret_cast<uint32_t(*)[16]>(r + N - 16));
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_cols(uint32_t taddr, const uint32_t *r) {
+  static_assert(N % 16 == 0, "16-column granularity");
+#pragma unroll
+  for (int c = 0; c + 32 <= N; c += 32)
+    tmem_st32(taddr + uint32_t(c), *reinterpret_cast<const uint32_t(*)[32]>(r + c));
+  if constexpr (N % 32 == 16)
+    tmem_st16(taddr + uint32_t(N - 16), *reinterpret_cast<const uint32_t(*)[16]>(r + N - 16));
+}
+
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory"); }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;\n" ::: "memory"); }
 

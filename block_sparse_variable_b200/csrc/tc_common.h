@@ -17,4 +17,11 @@ struct FwdMaps {
 
 cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m);
 
+// the backward also streams dOut with the q-tensor box
+struct BwdMaps {
+  CUtensorMap q, k, v, dout;
+};
+
+cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m);
+
 }  // namespace bsa

@@ -61,17 +61,30 @@ cudaError_t kv_map(CUtensorMap *m, const Problem &p, const void *base, int64_t s
   return encode(m, p, base, dims, strides, box);
 }
 
-}  // namespace
-
-cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m) {
+cudaError_t q_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb, int64_t sh,
+                  int64_t st) {
   const int64_t rows = p.q_layout == BSA_LAYOUT_TND ? p.Tq : p.Sq;
   const int64_t nb = p.q_layout == BSA_LAYOUT_TND ? 1 : p.B;
   const cuuint64_t dims[4] = {cuuint64_t(p.D), cuuint64_t(rows), cuuint64_t(p.N1), cuuint64_t(nb)};
-  const cuuint64_t strides[3] = {nz(p.q_st * 2), nz(p.q_sh * 2),
-                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * p.q_st * 2 : p.q_sb * 2)};
+  const cuuint64_t strides[3] = {nz(st * 2), nz(sh * 2),
+                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * st * 2 : sb * 2)};
   const cuuint32_t box[4] = {64, 128, 1, 1};
-  cudaError_t e = encode(&m.q, p, p.q, dims, strides, box);
+  return encode(m, p, base, dims, strides, box);
+}
+
+}  // namespace
+
+cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m) {
+  cudaError_t e = q_map(&m.q, p, p.q, p.q_sb, p.q_sh, p.q_st);
   if (e != cudaSuccess) return e;
+  if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
+  return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);
+}
+
+cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m) {
+  cudaError_t e = q_map(&m.q, p, p.q, p.q_sb, p.q_sh, p.q_st);
+  if (e != cudaSuccess) return e;
+  if ((e = q_map(&m.dout, p, p.dout, p.do_sb, p.do_sh, p.do_st)) != cudaSuccess) return e;
   if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
   return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);
 }

@@ -105,6 +105,7 @@ typedef enum bsa_status {
 #define BSA_FLAG_BAD_SEQLEN 0x2u  /* cu_seqlens / seqused_kv contradict the storage */
 #define BSA_FLAG_BAD_PAGE 0x4u    /* a block-table entry outside [0, num_pages) */
 #define BSA_FLAG_TIMEOUT 0x8u     /* a bounded device wait gave up (pipeline fault) */
+#define BSA_FLAG_INTERNAL 0x10u   /* a kernel precondition failed (internal error) */
 
 /* ------------------------------------------------------------- forward */
 /* Arguments:
