@@ -241,7 +241,7 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    p = workloads.make_config(args.config)
+    p = workloads.make_config(args.config, args.batch)
     pairs = _pairs(p)
     P = params_of(p)
     to = lambda t: None if t is None else t.to(dev)  # noqa: E731
@@ -269,6 +269,11 @@ def run_ours(args):
     flags = bsa.bsa_read_status(wsf) | bsa.bsa_read_status(wsb)
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # events the library records around each call's main attention kernel;
+    # they must exist on the device before their handles are passed on
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e in (e for row in kev for e in row):
+        e.record(stream)
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
@@ -277,8 +282,10 @@ def run_ours(args):
         start.record(stream)
         for s in range(args.steps):
             ev[s][0].record(stream)
+            bsa.bsa_set_main_kernel_events(kev[s][0], kev[s][1])
             bsa.bsa_fwd(q, k, v, index, P, out=out, lse=lse, workspace=wsf, stream=stream, **opt)
             ev[s][1].record(stream)
+            bsa.bsa_set_main_kernel_events(kev[s][2], kev[s][3])
             bsa.bsa_bwd(q, k, v, out, dout, lse, index, P, dq=dq, dk=dk, dv=dv, workspace=wsb,
                         stream=stream, **opt)
             ev[s][2].record(stream)
@@ -289,10 +296,12 @@ def run_ours(args):
     ms = start.elapsed_time(stop)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    fwd_kms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
+    bwd_kms = statistics.mean(e[2].elapsed_time(e[3]) for e in kev)
     if dist:
-        t = torch.tensor([ms, fwd_ms, bwd_ms], device=dev)
+        t = torch.tensor([ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms], device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, fwd_ms, bwd_ms = (float(x) for x in t.tolist())
+        ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms = (float(x) for x in t.tolist())
 
     # ---- end to end through the C ABI from pinned host buffers
     hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
@@ -337,23 +346,30 @@ def run_ours(args):
         value = world * step_flops / (ms_step * 1e-3) / 1e12
         fwd_tf = 4 * D * pairs / (fwd_ms * 1e-3) / 1e12
         bwd_tf = 10 * D * pairs / (bwd_ms * 1e-3) / 1e12
+        fwd_ktf = 4 * D * pairs / (fwd_kms * 1e-3) / 1e12
+        bwd_ktf = 10 * D * pairs / (bwd_kms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
-        dominant = "bwd" if bwd_ms >= fwd_ms else "fwd"
-        achieved = bwd_tf if dominant == "bwd" else fwd_tf
+        dominant = "bwd" if bwd_kms >= fwd_kms else "fwd"
+        achieved = bwd_ktf if dominant == "bwd" else fwd_ktf
         traffic = _traffic_from_profiles(args.config, dominant)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if p.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-            "config": {"workload": DESCR[args.config], "kept_pairs_per_replica": pairs,
+            "config": {"workload": DESCR[args.config] if args.batch is None
+                       else DESCR[args.config] + f" (batch overridden to {args.batch})",
+                       "kept_pairs_per_replica": pairs,
                        "parallelism": f"replicas x{world} (no exchange)",
                        "l2": "inputs larger than L2 (q/k/v/dout %d MiB each)"
                              % (q.numel() * q.element_size() >> 20)},
             "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
             "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
+            "kernel_ms": {"k_fwd_tc": round(fwd_kms, 4), "k_bwd_tc": round(bwd_kms, 4)},
+            "kernel_tflops": {"k_fwd_tc": round(fwd_ktf, 2), "k_bwd_tc": round(bwd_ktf, 2)},
             "pct_of_peak": round(100 * value / world / peak, 2),
-            "roofline": {"bound": "tensor", "kernel": f"bsa_{dominant} call (main kernel + prep)",
+            "roofline": {"bound": "tensor", "kernel": f"k_{dominant}_tc",
+                         "units": f"{10 if dominant == 'bwd' else 4}*D*kept_pairs FLOPs per launch",
                          "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_source": f"{which} bf16 burst",
                          "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
@@ -392,6 +408,8 @@ def main():
     ap.add_argument("--config", type=lambda s: int(s.lstrip("Cc")), default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="smaller batch for C3/C4 (profiler captures only; not a bench line)")
     args = ap.parse_args()
     if args.impl == "reference":
         run_reference(args)

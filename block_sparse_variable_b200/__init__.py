@@ -80,8 +80,10 @@ def _load():
     lib.bsa_status_string.argtypes = [ctypes.c_int]
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_abi_version.restype = ctypes.c_int32
+    lib.bsa_set_main_kernel_events.argtypes = [vp, vp]
     for f in ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_fwd_workspace_layout",
-              "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status"):
+              "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status",
+              "bsa_set_main_kernel_events"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -90,7 +92,8 @@ _lib = _load()
 
 EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bwd",
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
-            "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace")
+            "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace",
+            "bsa_set_main_kernel_events")
 
 
 def lib():
@@ -296,6 +299,15 @@ def bsa_read_status(workspace: torch.Tensor, stream=None) -> int:
 
 def bsa_status_string(status: int) -> str:
     return _lib.bsa_status_string(int(status)).decode()
+
+
+def bsa_set_main_kernel_events(before=None, after=None):
+    """The next bsa_fwd / bsa_bwd of this thread records the two
+    torch.cuda.Event objects around its main attention kernel (None, None
+    clears).  The events must already exist on the device: record each once
+    (on any stream) before handing it over."""
+    h = [None if e is None else ctypes.c_void_p(int(e.cuda_event)) for e in (before, after)]
+    _check(_lib.bsa_set_main_kernel_events(*h), "bsa_set_main_kernel_events")
 
 
 # ------------------------------------------------- forward without workspace

@@ -332,21 +332,35 @@ bsa_status check_ws(const Layout &L, void *ws, size_t bytes) {
     if ((x) != cudaSuccess) return BSA_ERR_CUDA; \
   } while (0)
 
-bsa_status run_fwd(const Problem &p, cudaStream_t s) {
+// events to record around the next call's main kernel (bsa_set_main_kernel_events)
+thread_local cudaEvent_t t_ev_before = nullptr, t_ev_after = nullptr;
+
+// takes the pending event pair of this host thread (at most one call uses it)
+void take_events(cudaEvent_t &before, cudaEvent_t &after) {
+  before = t_ev_before;
+  after = t_ev_after;
+  t_ev_before = t_ev_after = nullptr;
+}
+
+bsa_status run_fwd(const Problem &p, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   BSA_LAUNCH(bsa::launch_prep_geometry(p, s));
   BSA_LAUNCH(bsa::launch_prep_compact(p, true, s));
   BSA_LAUNCH(bsa::launch_sort_items(p, p.fwd_slots_pad, p.fwd_items, s));
+  if (e0) BSA_LAUNCH(cudaEventRecord(e0, s));
   BSA_LAUNCH(bsa::launch_fwd_main(p, s));
+  if (e1) BSA_LAUNCH(cudaEventRecord(e1, s));
   return BSA_OK;
 }
 
-bsa_status run_bwd(const Problem &p, cudaStream_t s) {
+bsa_status run_bwd(const Problem &p, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   BSA_LAUNCH(bsa::launch_prep_geometry(p, s));
   BSA_LAUNCH(bsa::launch_prep_compact(p, false, s));
   BSA_LAUNCH(bsa::launch_prep_inverse(p, s));
   BSA_LAUNCH(bsa::launch_sort_items(p, p.bwd_slots_pad, p.bwd_items, s));
   BSA_LAUNCH(bsa::launch_bwd_pre(p, s));
+  if (e0) BSA_LAUNCH(cudaEventRecord(e0, s));
   BSA_LAUNCH(bsa::launch_bwd_main(p, s));
+  if (e1) BSA_LAUNCH(cudaEventRecord(e1, s));
   BSA_LAUNCH(bsa::launch_bwd_post(p, s));
   return BSA_OK;
 }
@@ -374,6 +388,13 @@ Args bwd_args(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
 }  // namespace
 
 extern "C" {
+
+bsa_status bsa_set_main_kernel_events(void *before, void *after) {
+  if ((before == nullptr) != (after == nullptr)) return BSA_ERR_NULLPTR;
+  t_ev_before = static_cast<cudaEvent_t>(before);
+  t_ev_after = static_cast<cudaEvent_t>(after);
+  return BSA_OK;
+}
 
 int32_t bsa_abi_version(void) { return 1; }
 
@@ -423,6 +444,8 @@ bsa_status bsa_fwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
                    const bsa_tensor *seqused, const bsa_tensor *bt, const bsa_params *prm,
                    const bsa_tensor *out, const bsa_tensor *lse, void *workspace,
                    size_t workspace_bytes, void *stream) {
+  cudaEvent_t e0, e1;
+  take_events(e0, e1);
   Problem p;
   Layout L;
   bool empty;
@@ -430,7 +453,7 @@ bsa_status bsa_fwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
   if (st != BSA_OK || empty) return st;
   if ((st = check_ws(L, workspace, workspace_bytes)) != BSA_OK) return st;
   carve(p, L, workspace);
-  return run_fwd(p, static_cast<cudaStream_t>(stream));
+  return run_fwd(p, static_cast<cudaStream_t>(stream), e0, e1);
 }
 
 bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
@@ -473,6 +496,8 @@ bsa_status bsa_bwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
                    const bsa_tensor *seqused, const bsa_tensor *bt, const bsa_params *prm,
                    const bsa_tensor *dq, const bsa_tensor *dk, const bsa_tensor *dv,
                    void *workspace, size_t workspace_bytes, void *stream) {
+  cudaEvent_t e0, e1;
+  take_events(e0, e1);
   Problem p;
   Layout L;
   bool empty;
@@ -481,7 +506,7 @@ bsa_status bsa_bwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
   if (st != BSA_OK || empty) return st;
   if ((st = check_ws(L, workspace, workspace_bytes)) != BSA_OK) return st;
   carve(p, L, workspace);
-  return run_bwd(p, static_cast<cudaStream_t>(stream));
+  return run_bwd(p, static_cast<cudaStream_t>(stream), e0, e1);
 }
 
 bsa_status bsa_read_status(const void *workspace, void *stream, uint32_t *flags) {

@@ -18,12 +18,17 @@
 //     dV  += P^T dOut       (A from TMEM)
 //     dK  += dS^T Q         (A from TMEM)
 //     dQ_s = dS K           -> TMEM R1        (A = dS from shared memory)
-//   the softmax warps then add dQ_s (fp32) into the global dQ accumulator
-//   with vector reductions; after the item, dK * scale and dV are stored.
+//   the softmax warps then stage dQ_s (fp32) in shared memory over the
+//   step's Q and dOut tiles and the TMA warp has the TMA unit add it into the
+//   global dQ accumulator (bulk tensor reductions, which run on while the
+//   next steps compute); after the item, dK * scale and dV are stored.
 // TMEM columns: R0 [0,128), R1 [128,256), dV [256,256+D), dK [384,384+D).
+// Items of a kv head that share a query list start their walks at different
+// entries so that their dQ reductions do not meet on the same rows.
 // Warp roles (320 threads): 0..7 the two groups, 8 TMA (K, V per item; Q,
-// dOut per step into a 2-slot ring, with lse and Dsum staged by its lanes),
-// 9 TMEM owner and MMA issuer.  Every mbarrier wait is bounded.
+// dOut per step into a 2-slot ring, with lse and Dsum staged by its lanes;
+// the dQ reductions of the step that held a slot before), 9 TMEM owner and
+// MMA issuer.  Every mbarrier wait is bounded.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -49,15 +54,15 @@ enum : int {
   kBarKV = 0,       // K, V of the item landed
   kBarKVEmpty = 1,  // the item's MMAs are done with K, V
   kBarQD = 2,       // + slot: Q, dOut, lse, Dsum of a step landed
-  kBarQDEmpty = 4,  // + slot
-  kBarS = 6,        // S^T, dP^T of the step are in TMEM
-  kBarDS = 7,       // P, dS written (256 arrivals)
-  kBarP2 = 8,       // the step's dV, dK, dQ MMAs are done
-  kBarR1Free = 9,   // dQ of the step read out of TMEM (256 arrivals)
-  kBarAcc = 10,     // the item's dK, dV are final
-  kBarAccFree = 11, // dK, dV read out (256 arrivals)
-  kBarDrain = 12,
-  kNumBars = 13
+  kBarS = 4,        // S^T, dP^T of the step are in TMEM
+  kBarDS = 5,       // P, dS written (256 arrivals)
+  kBarP2 = 6,       // the step's dV, dK, dQ MMAs are done
+  kBarDQOut = 7,    // + slot: the step's dQ left TMEM and sits, staged, in
+                    // the slot's Q and dOut tiles (256 arrivals)
+  kBarAcc = 9,      // the item's dK, dV are final
+  kBarAccFree = 10, // dK, dV read out (256 arrivals)
+  kBarDrain = 11,
+  kNumBars = 12
 };
 
 template <int D>
@@ -78,7 +83,7 @@ struct BLayout {
 };
 
 struct BItem {
-  int b, h2, u0, kvlen, wb, pg, gk, steps_ok;
+  int b, h2, u0, kvlen, wb, pg, gk, steps_ok, rot;
   BatchInfo bi;
 };
 
@@ -95,6 +100,10 @@ __device__ __forceinline__ BItem b_item(const Problem &p, int id, int TK) {
   v.wb = min(128, v.bi.kvst - v.u0);
   v.pg = p.kv_layout == BSA_LAYOUT_PA_BBND ? kv_page(p, v.b, v.u0) : 0;
   v.steps_ok = v.pg >= 0;
+  // Items of one kv head that share a query list would otherwise walk it in
+  // the same order at the same time and pile their dQ reductions onto the
+  // same addresses; each starts at its own place in the list instead.
+  v.rot = v.gk * p.ksl + ks;
   return v;
 }
 
@@ -108,12 +117,19 @@ __device__ __forceinline__ int64_t b_list(const Problem &p, const BItem &v, int 
   return int64_t(hi) * TK + v.gk;
 }
 
+// q block of entry e (in walking order) of the item's list for q head hh
+__device__ __forceinline__ int b_qblock(const Problem &p, const BItem &v, int hh, int e, int TK) {
+  const int64_t li = b_list(p, v, hh, TK);
+  const int off = p.inv_off[li], len = p.inv_off[li + 1] - off;
+  return p.inv_list[off + (e + v.rot) % len];
+}
+
 __device__ __forceinline__ BStep b_settle(const Problem &p, const BItem &v, BStep c, int TK) {
   while (c.hh < p.g) {
     const int64_t li = b_list(p, v, c.hh, TK);
     const int len = p.inv_off[li + 1] - p.inv_off[li];
     if (c.e < len) {
-      const int i = p.inv_list[p.inv_off[li] + c.e];
+      const int i = p.inv_list[p.inv_off[li] + (c.e + v.rot) % len];
       if (c.st < p.nsub && i * p.BQ + c.st * 128 < v.bi.qlen) return c;
       ++c.e;
       c.st = 0;
@@ -132,20 +148,14 @@ __device__ __forceinline__ BStep b_next(const Problem &p, const BItem &v, BStep 
 }
 
 __device__ __forceinline__ int b_t0(const Problem &p, const BItem &v, const BStep &c, int TK) {
-  return p.inv_list[p.inv_off[b_list(p, v, c.hh, TK)] + c.e] * p.BQ + c.st * 128;
-}
-
-__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"l"(addr), "f"(a), "f"(b),
-               "f"(c), "f"(d)
-               : "memory");
+  return b_qblock(p, v, c.hh, c.e, TK) * p.BQ + c.st * 128;
 }
 
 template <int D, bool BF16>
 __global__ void __launch_bounds__(kBThreads, 1)
     k_bwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-             const __grid_constant__ CUtensorMap map_do) {
+             const __grid_constant__ CUtensorMap map_do, const __grid_constant__ CUtensorMap map_dq) {
   using L = BLayout<D>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ unsigned char smem_raw[];
@@ -171,12 +181,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kBarKVEmpty), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarQD + s), 1);
-      mbar_init(bar(kBarQDEmpty + s), 1);
+      mbar_init(bar(kBarDQOut + s), 256);
     }
     mbar_init(bar(kBarS), 1);
     mbar_init(bar(kBarDS), 256);
     mbar_init(bar(kBarP2), 1);
-    mbar_init(bar(kBarR1Free), 256);
     mbar_init(bar(kBarAcc), 1);
     mbar_init(bar(kBarAccFree), 256);
     mbar_init(bar(kBarDrain), 1);
@@ -201,10 +210,32 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tma_prefetch_desc(&map_k);
       tma_prefetch_desc(&map_v);
       tma_prefetch_desc(&map_do);
+      tma_prefetch_desc(&map_dq);
     }
     uint32_t kv_it = 0, sk = 0;
     int armed_kv = -1, armed_qd[2] = {-1, -1};
+    int pend_row[2] = {0, 0}, pend_h[2] = {0, 0};  // dQ origin of the step held in each slot
     bool ok = true;
+    // A step is done with its slot once its dQ, staged there by the softmax
+    // warps, has been handed to the TMA unit and read back out of shared
+    // memory; the additions into global memory then proceed on their own.
+    // One commit group per tile: the Q tile's boxes, then the dOut tile's.
+    auto reduce_slot = [&](int sl) {
+#pragma unroll
+      for (int j = 0; j < D / 32; ++j) {
+        const uint32_t src = j < D / 64 ? sQ + sl * L::kTile + j * L::kBox
+                                        : sDO + sl * L::kTile + (j - D / 64) * L::kBox;
+        tma_reduce_add_3d(&map_dq, src, 32 * j, pend_h[sl], pend_row[sl]);
+        if (j == D / 64 - 1 || j == D / 32 - 1) bulk_commit();
+      }
+    };
+    auto flush = [&](uint32_t s) -> bool {  // the last two steps, after the loop
+      const int sl = int(s & 1u);
+      if (!wait_warp(bar(kBarDQOut + sl), (s >> 1) & 1u, abort, p.status)) return false;
+      if (lane == 0) reduce_slot(sl);
+      __syncwarp();
+      return true;
+    };
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) continue;
@@ -224,44 +255,62 @@ __global__ void __launch_bounds__(kBThreads, 1)
       ++kv_it;
       for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
         const int slot = int(sk & 1u);
-        if (!(ok = wait_warp(bar(kBarQDEmpty + slot), ((sk >> 1) & 1u) ^ 1u, abort, p.status))) break;
         const int h1 = v.h2 * p.g + c.hh;
         const int t0 = b_t0(p, v, c, TK);
-        // lse (log2 units) and Dsum of the step's 128 query rows; rows past
-        // qlen get lse = +inf (so P = 0) and Dsum = 0
-        float *st = stat + slot * 256;
-        for (int j = lane; j < 128; j += 32) {
-          const int t = t0 + j;
-          float l2 = INFINITY, ds = 0.f;
+        // lse (log2 units) and Dsum of the step's 128 query rows, fetched
+        // before waiting for the slot; rows past qlen get lse = +inf (so
+        // P = 0) and Dsum = 0
+        float l2r[4], dsr[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = t0 + lane + 32 * i;
+          l2r[i] = INFINITY;
+          dsr[i] = 0.f;
           if (t < v.bi.qlen) {
-            l2 = p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, h1, t)] * kLog2e;
-            if (!(l2 > -INFINITY)) l2 = INFINITY;  // a row with no selected key
+            const float l2 = p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, h1, t)] * kLog2e;
+            l2r[i] = l2 > -INFINITY ? l2 : INFINITY;  // a row with no selected key
             const int64_t srow = p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq + t : v.bi.q_tok0 + t;
-            ds = p.dsum[srow * p.N1 + h1];
+            dsr[i] = p.dsum[srow * p.N1 + h1];
           }
-          st[j] = l2;
-          st[128 + j] = ds;
+        }
+        // the step that held the slot before: its dQ is staged over the
+        // slot's tiles; hand it to the TMA unit in two commit groups (Q tile,
+        // dOut tile) so that each tile is refilled as soon as it is read out
+        const bool refill = sk >= 2;
+        if (refill && !(ok = wait_warp(bar(kBarDQOut + slot), ((sk - 2) >> 1) & 1u, abort, p.status))) break;
+        float *st = stat + slot * 256;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          st[lane + 32 * i] = l2r[i];
+          st[128 + lane + 32 * i] = dsr[i];
         }
         __syncwarp();
         if (lane == 0) {
+          if (refill) reduce_slot(slot);
           mbar_expect_tx(bar(kBarQD + slot), 2 * L::kTile);
           armed_qd[slot] = int((sk >> 1) & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
-          for (int h = 0; h < D / 64; ++h) {
+          if (refill) bulk_wait_read<1>();
+          for (int h = 0; h < D / 64; ++h)
             tma_load_4d(sQ + slot * L::kTile + h * L::kBox, &map_q, bar(kBarQD + slot), h * 64, tok, h1, bb);
+          if (refill) bulk_wait_read<0>();
+          for (int h = 0; h < D / 64; ++h)
             tma_load_4d(sDO + slot * L::kTile + h * L::kBox, &map_do, bar(kBarQD + slot), h * 64, tok, h1, bb);
-          }
         }
         __syncwarp();
+        pend_h[slot] = h1;
+        pend_row[slot] = int((p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq : v.bi.q_tok0) + t0);
         ++sk;
       }
     }
+    for (uint32_t s = sk >= 2 ? sk - 2 : 0; s < sk && ok; ++s) ok = flush(s);
     if (*abort && lane == 0) {  // let every copy already issued land before the CTA exits
       if (armed_kv >= 0) drain_wait(bar(kBarKV), uint32_t(armed_kv));
       for (int s = 0; s < 2; ++s)
         if (armed_qd[s] >= 0) drain_wait(bar(kBarQD + s), uint32_t(armed_qd[s]));
     }
+    if (lane == 0) bulk_wait_all();  // every dQ addition has been made
   } else if (warp == kBMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     constexpr uint32_t idSP = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
@@ -298,7 +347,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const int slot = int(sk & 1u);
         if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
         // R1 still holds the previous step's dQ until it has been read out
-        if (sk > 0 && !(ok = wait_warp(bar(kBarR1Free), (sk - 1) & 1u, abort, p.status))) break;
+        if (sk > 0 && !(ok = wait_warp(bar(kBarDQOut + ((sk - 1) & 1u)), ((sk - 1) >> 1) & 1u, abort, p.status)))
+          break;
         tc_fence_after();
         const uint64_t dQk = sw128_desc(sQ + slot * L::kTile, 16, 1024);
         const uint64_t dOk = sw128_desc(sDO + slot * L::kTile, 16, 1024);
@@ -325,7 +375,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
             mma_ss(tR1, dDS + uint64_t(kk * 128), dKmn + uint64_t(kk * 128), idQ, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(kBarP2));
-          mma_commit(bar(kBarQDEmpty + slot));
         }
         __syncwarp();
         first = false;
@@ -346,7 +395,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   } else {
     // ------------------------------------------- the two softmax groups
     const int wg = warp >> 2;
-    const int r = tid & 127;  // kv row (phase 1 / epilogue) or q row (dQ read-out)
+    const int r = tid & 127;  // kv row (TMEM lane) of the softmax and the epilogue
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     uint32_t sk = 0, item_n = 0;
     bool ok = true;
@@ -360,7 +409,6 @@ __global__ void __launch_bounds__(kBThreads, 1)
       int nsteps = 0;
       for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
         const int slot = int(sk & 1u);
-        const int h1 = v.h2 * p.g + c.hh;
         const int t0 = b_t0(p, v, c, TK);
         if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
         if (!(ok = wait_warp(bar(kBarS), sk & 1u, abort, p.status))) break;
@@ -401,29 +449,32 @@ __global__ void __launch_bounds__(kBThreads, 1)
         fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kBarDS));
-        // dQ of the step (lanes = q rows): add into the fp32 accumulator
+        // dQ of the step (TMEM lanes = q rows) out to shared memory, where the
+        // step's Q and dOut tiles were (free once its MMAs are done): four
+        // boxes of 32 fp32 columns x 128 rows in the 128-byte swizzle, group
+        // 0's in the Q tile and group 1's in the dOut tile.  The TMA warp adds
+        // them into the global accumulator.  Rows past qlen are staged as
+        // zeros: adding them changes nothing.
         if (!(ok = wait_warp(bar(kBarP2), sk & 1u, abort, p.status))) break;
         tc_fence_after();
         {
-          const int t = t0 + r;
-          const bool q_ok = t < v.bi.qlen;
-          const int64_t srow = p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq + t : v.bi.q_tok0 + t;
-          float *dq = p.dq_acc + (srow * p.N1 + h1) * D + (D / 2) * wg;
+          const bool q_ok = t0 + r < v.bi.qlen;
+          unsigned char *boxes = sbase + (wg == 0 ? L::kQ : L::kDO) + slot * L::kTile;
 #pragma unroll
           for (int h = 0; h < D / 64; ++h) {
             uint32_t x[32];
             tmem_ld32(tR1 + lane_off + uint32_t((D / 2) * wg + 32 * h), x);
             tmem_wait_ld();
-            if (q_ok) {
+            uint4 *row = reinterpret_cast<uint4 *>(boxes + h * L::kBox + r * 128);
 #pragma unroll
-              for (int c = 0; c < 32; c += 4)
-                red_add_v4(dq + 32 * h + c, __uint_as_float(x[c]), __uint_as_float(x[c + 1]),
-                           __uint_as_float(x[c + 2]), __uint_as_float(x[c + 3]));
-            }
+            for (int c = 0; c < 8; ++c)
+              row[c ^ (r & 7)] = q_ok ? make_uint4(x[4 * c], x[4 * c + 1], x[4 * c + 2], x[4 * c + 3])
+                                      : make_uint4(0, 0, 0, 0);
           }
         }
+        fence_proxy_async_smem();
         tc_fence_before();
-        mbar_arrive(bar(kBarR1Free));
+        mbar_arrive(bar(kBarDQOut + slot));
         ++sk;
         ++nsteps;
       }
@@ -490,7 +541,7 @@ cudaError_t launch_bwd_tc(const Problem &p, const BwdMaps &m, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t grid = p.bwd_slots < num_sms() ? p.bwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_bwd_tc<D, BF16><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout);
+  k_bwd_tc<D, BF16><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
   return cudaGetLastError();
 }
 

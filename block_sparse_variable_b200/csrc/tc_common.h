@@ -17,9 +17,11 @@ struct FwdMaps {
 
 cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m);
 
-// the backward also streams dOut with the q-tensor box
+// the backward also streams dOut with the q-tensor box, and adds its dQ
+// tiles into the fp32 accumulator [rows][N1][D] through a 3-D map
+// {D, N1, rows} with 32-column x 1-head x 128-row boxes (128-byte swizzle)
 struct BwdMaps {
-  CUtensorMap q, k, v, dout;
+  CUtensorMap q, k, v, dout, dq_acc;
 };
 
 cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m);

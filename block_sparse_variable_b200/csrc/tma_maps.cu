@@ -42,6 +42,19 @@ cudaError_t encode(CUtensorMap *m, const Problem &p, const void *base, const cuu
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+cudaError_t dq_acc_map(CUtensorMap *m, const Problem &p) {
+  EncodeTiled fn = encoder();
+  if (!fn) return cudaErrorNotSupported;
+  const cuuint64_t dims[3] = {cuuint64_t(p.D), cuuint64_t(p.N1), cuuint64_t(p.rows_q)};
+  const cuuint64_t strides[2] = {cuuint64_t(p.D) * 4, cuuint64_t(p.N1) * p.D * 4};
+  const cuuint32_t box[3] = {32, 1, 128};
+  const cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, p.dq_acc, dims, strides, box, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cuuint64_t nz(int64_t x) { return x > 0 ? cuuint64_t(x) : 16; }
 
 cudaError_t kv_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb, int64_t sh,
@@ -86,7 +99,8 @@ cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m) {
   if (e != cudaSuccess) return e;
   if ((e = q_map(&m.dout, p, p.dout, p.do_sb, p.do_sh, p.do_st)) != cudaSuccess) return e;
   if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
-  return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);
+  if ((e = kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st)) != cudaSuccess) return e;
+  return dq_acc_map(&m.dq_acc, p);
 }
 
 }  // namespace bsa

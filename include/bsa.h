@@ -253,6 +253,17 @@ bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, co
                                     const bsa_tensor *dk, const bsa_tensor *dv,
                                     bsa_ws_layout *layout);
 
+/* Profiling hook (the pages have no counterpart).  The next bsa_fwd or
+ * bsa_bwd call made by this host thread records `before` and `after`
+ * (cudaEvent_t handles created by the caller, passed as void*) on its stream
+ * immediately before and after its main attention kernel, so that kernel's
+ * duration can be timed apart from the preparation kernels; the setting is
+ * then cleared, whatever the call's outcome: a call that launches nothing
+ * (failed validation, an empty problem) records nothing.  Both NULL clears a
+ * pending pair; exactly one NULL returns BSA_ERR_NULLPTR.  bsa_fwd_static_
+ * workspace passes the pair on to its bsa_fwd. */
+bsa_status bsa_set_main_kernel_events(void *before, void *after);
+
 /* Library ABI version (bumped on any signature or layout change). */
 int32_t bsa_abi_version(void);
 

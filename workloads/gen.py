@@ -235,8 +235,13 @@ def _lens(seed, B, lo, hi):
     return [int(x) for x in rng.integers(lo, hi + 1, size=B)]
 
 
-def make_config(c: int) -> Problem:
-    """C1..C5: the five workload shapes (see the module docstring for seeds)."""
+def make_config(c: int, batch: int | None = None) -> Problem:
+    """C1..C5: the five workload shapes (see the module docstring for seeds).
+
+    `batch` overrides the batch of the BNSD shapes C3 and C4 (smaller cases
+    of the same kernels for profiler captures)."""
+    if batch is not None and c not in (3, 4):
+        raise ValueError("batch override applies to C3 and C4 only")
     s = 1000 * c
     if c == 1:
         return make_problem(name="C1", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=64,
@@ -248,10 +253,10 @@ def make_config(c: int) -> Problem:
                             pattern=pat_fraction_diag(0.25), W=max(math.ceil(l / 128) for l in lens),
                             seed_base=s)
     if c == 3:
-        return make_problem(name="C3", layout_q="BNSD", layout_kv="BNSD", B=2, N1=32, N2=32, D=128,
+        return make_problem(name="C3", layout_q="BNSD", layout_kv="BNSD", B=batch or 2, N1=32, N2=32, D=128,
                             Sq=8192, BQ=128, BKV=512, W=16, pattern=pat_dense, seed_base=s)
     if c == 4:
-        return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=1, N1=24, N2=24, D=128,
+        return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=batch or 1, N1=24, N2=24, D=128,
                             Sq=32768, BQ=128, BKV=128, W=256, pattern=pat_sink_diag_random(14),
                             seed_base=s)
     if c == 5:
