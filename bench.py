@@ -221,6 +221,23 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+# ------------------------------------------------------------ rank plumbing
+def max_over_ranks(dist, values, device):
+    """Element-wise maximum of per-rank timings (the slowest rank sets the
+    time); identity without a process group."""
+    if dist is None:
+        return [float(x) for x in values]
+    t = torch.tensor([float(x) for x in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
+def job_tflops(world, flops_per_replica_step, ms_per_step):
+    """Whole-job throughput: every rank runs one replica of the step, so the
+    job does world x the work in the slowest rank's time."""
+    return world * flops_per_replica_step / (ms_per_step * 1e-3) / 1e12
+
+
 # -------------------------------------------------------------------- GPU leg
 def run_ours(args):
     import block_sparse_variable_b200 as bsa
@@ -298,10 +315,7 @@ def run_ours(args):
     bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
     fwd_kms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
     bwd_kms = statistics.mean(e[2].elapsed_time(e[3]) for e in kev)
-    if dist:
-        t = torch.tensor([ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms = (float(x) for x in t.tolist())
+    ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms = max_over_ranks(dist, [ms, fwd_ms, bwd_ms, fwd_kms, bwd_kms], dev)
 
     # ---- end to end through the C ABI from pinned host buffers
     hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, dout))
@@ -332,18 +346,14 @@ def run_ours(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms, = max_over_ranks(dist, [e0.elapsed_time(e1) / e2e_steps], dev)
 
     if rank == 0:
         peaks, which = _peaks()
         D = p.D
         step_flops = 14 * D * pairs
         ms_step = ms / args.steps
-        value = world * step_flops / (ms_step * 1e-3) / 1e12
+        value = job_tflops(world, step_flops, ms_step)
         fwd_tf = 4 * D * pairs / (fwd_ms * 1e-3) / 1e12
         bwd_tf = 10 * D * pairs / (bwd_ms * 1e-3) / 1e12
         fwd_ktf = 4 * D * pairs / (fwd_kms * 1e-3) / 1e12
@@ -374,7 +384,7 @@ def run_ours(args):
                          "frac": round(achieved / peak, 4), "peak_source": f"{which} bf16 burst",
                          "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
                          "traffic": traffic},
-            "e2e": {"value": round(world * step_flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "e2e": {"value": round(job_tflops(world, step_flops, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
             "gpu_launches": LAUNCHES_PER_STEP * args.steps,
