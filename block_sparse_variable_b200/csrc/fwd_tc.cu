@@ -69,9 +69,10 @@ enum : int {
   kBarSFull = 14,   // + S buffer
   kBarPFull = 17,   // + S buffer (one arrival per softmax thread)
   kBarPVDone = 20,  // + (chunk index & 1): P_t V_t is in O
-  kBarXchg = 22,    // the softmax groups' rendezvous (one arrival per softmax thread)
-  kBarDrain = 23,
-  kNumBars = 24
+  kBarXchg = 22,    // + row quarter: rendezvous of the warps that share 32 query
+                    // rows (one per group; 32 arrivals per warp)
+  kBarDrain = 26,
+  kNumBars = 27
 };
 
 template <int D>
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(bar(kBarPVDone), 1);
     mbar_init(bar(kBarPVDone + 1), 1);
-    mbar_init(bar(kBarXchg), kSoftmaxThreads);
+    for (int q = 0; q < 4; ++q) mbar_init(bar(kBarXchg + q), kSoftmaxThreads / 4);
     mbar_init(bar(kBarDrain), 1);
     *abort = 0;
     fence_barrier_init();
@@ -261,73 +262,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint64_t dK = sw128_desc(sK, 16, 1024);
     const uint64_t dV = sw128_desc(sV, L::kBox, 1024);
     auto kstep = [](int kk) { return uint64_t((kk >> 2) * (L::kBox >> 4) + (kk & 3) * 2); };
+    // 16 kv columns of P = 8 TMEM columns; the first 64 kv columns' P is in
+    // TMEM columns [0, 32), the next 64's in [64, 96) of the S buffer
+    auto pcol = [](int kk) { return uint32_t(64 * (kk >> 2) + 8 * (kk & 3)); };
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
     // Issue P_pv V_pv (pv >= 0) interleaved with S_sa, S_sb (>= 0), then
     // signal: S_full / K_empty per S, PV_done / V_empty for the product,
-    // Q_empty after the item's last S (last_s).
-    auto issue = [&](int64_t pv, bool pv_first, int pv_valid, int64_t sa, int64_t sb,
-                     int64_t last_s) {
+    // Q_empty after the item's last S (last_s).  One thread does all of it:
+    // the waits are single-thread polls, nothing warp-collective on the path.
+    auto issue = [&](int64_t pv, bool pv_first, int64_t sa, int64_t sb, int64_t last_s) {
+      if (sa >= 0 && !(ok = wait_bar(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
+      if (sb >= 0 && !(ok = wait_bar(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
       if (pv >= 0) {
-        if (!(ok = wait_warp(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
-        if (!(ok = wait_warp(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
-        if (p.kv_layout == BSA_LAYOUT_PA_BBND && pv_valid < 128) {
-          // rows of the last page past the used length may hold anything
-          // (even NaN); their P is 0, so make their V exactly 0 as well
-          uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + int(pv % kStages) * L::kTile);
-          const int per_half = (128 - pv_valid) * 8;  // 16-byte words per 64-column half
-          for (int w = lane; w < per_half * (D / 64); w += 32) {
-            const int h = w / per_half, x = w % per_half;
-            vt[h * (L::kBox / 16) + pv_valid * 8 + x] = make_uint4(0, 0, 0, 0);
-          }
-          fence_proxy_async_smem();
-          __syncwarp();
-        }
+        if (!(ok = wait_bar(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
+        // P_pv written (and, for a partial paged chunk, the V rows past the
+        // used length zeroed by the softmax warps)
+        if (!(ok = wait_bar(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
       }
-      if (sa >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
-      if (sb >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
       tc_fence_after();
-      if (lane == 0) {
-        const uint32_t pa = tS0 + uint32_t(pv % kSBufs) * 128u;
-        const uint64_t vd = dV + uint64_t((pv % kStages) * (L::kTile >> 4));
-        const uint32_t da = tS0 + uint32_t(sa % kSBufs) * 128u, db = tS0 + uint32_t(sb % kSBufs) * 128u;
-        const uint64_t ka = dK + uint64_t((sa % kStages) * (L::kTile >> 4));
-        const uint64_t kb = dK + uint64_t((sb % kStages) * (L::kTile >> 4));
+      const uint32_t pa = tS0 + uint32_t(pv % kSBufs) * 128u;
+      const uint64_t vd = dV + uint64_t((pv % kStages) * (L::kTile >> 4));
+      const uint32_t da = tS0 + uint32_t(sa % kSBufs) * 128u, db = tS0 + uint32_t(sb % kSBufs) * 128u;
+      const uint64_t ka = dK + uint64_t((sa % kStages) * (L::kTile >> 4));
+      const uint64_t kb = dK + uint64_t((sb % kStages) * (L::kTile >> 4));
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          if (pv >= 0)
-            mma_ts(tO, pa + uint32_t(kk) * 8u, vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
-          if (kk < D / 16) {
-            if (sa >= 0) mma_ss(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
-            if (sb >= 0) mma_ss(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
-          }
+      for (int kk = 0; kk < 8; ++kk) {
+        if (pv >= 0)
+          mma_ts(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
+        if (kk < D / 16) {
+          if (sa >= 0) mma_ss(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          if (sb >= 0) mma_ss(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
         }
-        if (sa >= 0) { mma_commit(bar(kBarSFull + int(sa % kSBufs))); mma_commit(bar(kBarKEmpty + int(sa % kStages))); }
-        if (sb >= 0) { mma_commit(bar(kBarSFull + int(sb % kSBufs))); mma_commit(bar(kBarKEmpty + int(sb % kStages))); }
-        if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit(bar(kBarQEmpty));
-        if (pv >= 0) { mma_commit(bar(kBarPVDone + int(pv & 1))); mma_commit(bar(kBarVEmpty + int(pv % kStages))); }
       }
-      __syncwarp();
+      if (sa >= 0) { mma_commit(bar(kBarSFull + int(sa % kSBufs))); mma_commit(bar(kBarKEmpty + int(sa % kStages))); }
+      if (sb >= 0) { mma_commit(bar(kBarSFull + int(sb % kSBufs))); mma_commit(bar(kBarKEmpty + int(sb % kStages))); }
+      if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit(bar(kBarQEmpty));
+      if (pv >= 0) { mma_commit(bar(kBarPVDone + int(pv & 1))); mma_commit(bar(kBarVEmpty + int(pv % kStages))); }
     };
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const ItemView v = item_view(p, p.fwd_items[it]);
-      const int n = count_chunks(p, v);
-      if (n == 0) continue;
-      if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
-      ++q_it;
-      const int64_t t0 = kv_it, last = kv_it + n - 1;
-      issue(-1, false, 128, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
-      Chunk ch = settle(p, v, Chunk{0, 0});
-      for (int j = 0; j < n && ok; ++j) {
-        const int valid = v.kvlen - v.u0(ch);
-        issue(t0 + j, j == 0, valid, j + 2 < n ? t0 + j + 2 : -1, -1, last);
-        ch = next_chunk(p, v, ch);
+    if (lane == 0) {
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+        const ItemView v = item_view(p, p.fwd_items[it]);
+        const int n = count_chunks(p, v);
+        if (n == 0) continue;
+        if (!(ok = wait_bar(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
+        ++q_it;
+        const int64_t t0 = kv_it, last = kv_it + n - 1;
+        issue(-1, false, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
+        for (int j = 0; j < n && ok; ++j) issue(t0 + j, j == 0, j + 2 < n ? t0 + j + 2 : -1, -1, last);
+        kv_it += uint32_t(n);
       }
-      kv_it += uint32_t(n);
-    }
-    if (*abort && lane == 0) {  // let issued MMAs finish before TMEM is freed
-      mma_commit(bar(kBarDrain));
-      drain_wait(bar(kBarDrain), 0);
+      if (*abort) {  // let issued MMAs finish before TMEM is freed
+        mma_commit(bar(kBarDrain));
+        drain_wait(bar(kBarDrain), 0);
+      }
     }
     __syncwarp();
   } else if (warp < kLoadWarp) {
@@ -341,10 +329,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     constexpr int kWarps = 4 * kSoftmaxGroups;
     uint32_t kv_it = 0, x_it = 0;  // global chunk counter; rendezvous counter
     bool ok = true;
-    // all softmax threads meet here (bounded: an aborted peer cannot strand us)
+    // the warps holding the same 32 query rows (one per group) meet here
+    // (bounded: an aborted peer cannot strand us)
     auto rendezvous = [&]() {
-      mbar_arrive(bar(kBarXchg));
-      ok = wait_warp(bar(kBarXchg), x_it & 1u, abort, p.status);
+      mbar_arrive(bar(kBarXchg + (warp & 3)));
+      ok = wait_warp(bar(kBarXchg + (warp & 3)), x_it & 1u, abort, p.status);
       ++x_it;
       return ok;
     };
@@ -372,6 +361,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t tS = tS0 + uint32_t(b) * 128u + lane_off;
           const int valid_all = v.kvlen - v.u0(ch);       // kv columns of the chunk that exist
           const int valid = valid_all - kCols * wg;        // of this group's columns
+          if (p.kv_layout == BSA_LAYOUT_PA_BBND && valid_all < 128) {
+            // rows of the last page past the used length may hold anything
+            // (even NaN); their P is 0, so make their V exactly 0 as well
+            // (before P is published: the MMA reads V after P_full)
+            const int st = int(kv_it % kStages);
+            if (!(ok = wait_warp(bar(kBarVFull + st), (kv_it / kStages) & 1u, abort, p.status))) break;
+            uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + st * L::kTile);
+            const int per_half = (128 - valid_all) * 8;  // 16-byte words per 64-column half
+            for (int w = tid; w < per_half * (D / 64); w += kSoftmaxThreads) {
+              const int h = w / per_half, x = w % per_half;
+              vt[h * (L::kBox / 16) + valid_all * 8 + x] = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+          }
           uint32_t x[kCols];
           tmem_ld_cols<kCols>(tS + uint32_t(kCols * wg), x);
           tmem_wait_ld();
@@ -388,13 +391,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const bool first = m == -INFINITY;
           const uint32_t need = __any_sync(0xffffffffu, first || hmax > m + kRescaleThreshold) ? 1u : 0u;
           if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
-          // after this rendezvous every S column has been read: P may overwrite S
           if (!rendezvous()) break;
-          // one decision for the whole CTA, so that every group takes the
-          // same number of rendezvous
+          // one decision for the rows of this warp, shared with the other
+          // group's warp on the same rows, so that both take the same path
           uint32_t any = 0;
 #pragma unroll
-          for (int w = 0; w < kWarps; ++w) any |= flags[(kv_it & 1u) * kWarps + w];
+          for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) any |= flags[(kv_it & 1u) * kWarps + 4 * g2 + (warp & 3)];
           float alpha = 1.f;
           const bool grow = any != 0u;
           if (grow) {
@@ -429,7 +431,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ps[(c >> 1) & 1] += e0 + e1;
             pk[c >> 1] = MmaOp<T>::pack(e0, e1);
           }
-          tmem_st_cols<kCols / 2>(tS + uint32_t((kCols / 2) * wg), pk);
+          // P over the first half of this group's own S columns: no other
+          // warp reads them any more (the grow path's reads of the other
+          // group's S precede its rendezvous)
+          tmem_st_cols<kCols / 2>(tS + uint32_t(kCols * wg), pk);
           l = l * alpha + (ps[0] + ps[1]);
           if (grow && !first && __any_sync(0xffffffffu, alpha != 1.f)) {
             // O may only be rescaled once P_{t-1} V_{t-1} (and so every
