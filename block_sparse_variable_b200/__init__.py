@@ -81,9 +81,10 @@ def _load():
     lib.bsa_status_string.restype = ctypes.c_char_p
     lib.bsa_abi_version.restype = ctypes.c_int32
     lib.bsa_set_main_kernel_events.argtypes = [vp, vp]
+    lib.bsa_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
     for f in ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_fwd_workspace_layout",
               "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status",
-              "bsa_set_main_kernel_events"):
+              "bsa_set_main_kernel_events", "bsa_selftest_exp2"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -93,7 +94,7 @@ _lib = _load()
 EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bwd",
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
             "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace",
-            "bsa_set_main_kernel_events")
+            "bsa_set_main_kernel_events", "bsa_selftest_exp2")
 
 
 def lib():
@@ -299,6 +300,17 @@ def bsa_read_status(workspace: torch.Tensor, stream=None) -> int:
 
 def bsa_status_string(status: int) -> str:
     return _lib.bsa_status_string(int(status)).decode()
+
+
+def bsa_selftest_exp2(x: torch.Tensor, stream=None):
+    """(FMA-pipe 2^x of the softmax kernels, hardware ex2.approx) of a CUDA
+    float32 tensor, elementwise."""
+    x = x.contiguous()
+    yp, ym = torch.empty_like(x), torch.empty_like(x)
+    _check(_lib.bsa_selftest_exp2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(yp.data_ptr()),
+                                  ctypes.c_void_p(ym.data_ptr()), x.numel(),
+                                  ctypes.c_void_p(_stream(stream))), "bsa_selftest_exp2")
+    return yp, ym
 
 
 def bsa_set_main_kernel_events(before=None, after=None):

@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     };
     auto flush = [&](uint32_t s) -> bool {  // the last two steps, after the loop
       const int sl = int(s & 1u);
-      if (!wait_warp(bar(kBarDQOut + sl), (s >> 1) & 1u, abort, p.status)) return false;
+      if (!wait_warp_lazy(bar(kBarDQOut + sl), (s >> 1) & 1u, abort, p.status)) return false;
       if (lane == 0) reduce_slot(sl);
       __syncwarp();
       return true;
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) continue;
-      if (!(ok = wait_warp(bar(kBarKVEmpty), (kv_it & 1u) ^ 1u, abort, p.status))) break;
+      if (!(ok = wait_warp_lazy(bar(kBarKVEmpty), (kv_it & 1u) ^ 1u, abort, p.status))) break;
       if (lane == 0) {
         mbar_expect_tx(bar(kBarKV), 2 * L::kTile);
         armed_kv = int(kv_it & 1u);
@@ -277,7 +277,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         // slot's tiles; hand it to the TMA unit in two commit groups (Q tile,
         // dOut tile) so that each tile is refilled as soon as it is read out
         const bool refill = sk >= 2;
-        if (refill && !(ok = wait_warp(bar(kBarDQOut + slot), ((sk - 2) >> 1) & 1u, abort, p.status))) break;
+        if (refill && !(ok = wait_warp_lazy(bar(kBarDQOut + slot), ((sk - 2) >> 1) & 1u, abort, p.status))) break;
         float *st = stat + slot * 256;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {

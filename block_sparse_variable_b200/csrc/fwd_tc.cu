@@ -37,6 +37,7 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
+#include "exp2_poly.cuh"
 #include "ptx_sm80.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -57,6 +58,9 @@ constexpr int kMmaWarp = kLoadWarp + 1;
 constexpr int kVLoadWarp = kLoadWarp + 2;
 constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+// of every 8 column pairs, this many take their exponentials on the FMA pipe
+// (exp2_poly) instead of the MUFU unit, which alone would bound the softmax
+constexpr int kPolyPairsOf8 = 0;
 
 // barrier slots
 enum : int {
@@ -218,7 +222,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const ItemView v = item_view(p, p.fwd_items[it]);
         if (count_chunks(p, v) == 0) continue;
         if (is_k) {
-          if (!(ok = wait_bar(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status))) break;
+          if (!(ok = wait_bar_lazy(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status))) break;
           mbar_expect_tx(bar(kBarQFull), L::kTile);
           armed_q = int(q_it & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + v.t0 : v.t0;
@@ -237,7 +241,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (p.kv_layout == BSA_LAYOUT_PA_BBND) { c1 = v.h2; c2 = u0 % p.page_size; c3 = pg; }
           else if (p.kv_layout == BSA_LAYOUT_TND) { c1 = int(v.bi.kv_tok0) + u0; c2 = v.h2; c3 = 0; }
           else { c1 = u0; c2 = v.h2; c3 = v.b; }
-          if (!(ok = wait_bar(bar(empty0 + s), ph ^ 1u, abort, p.status))) break;
+          if (!(ok = wait_bar_lazy(bar(empty0 + s), ph ^ 1u, abort, p.status))) break;
           mbar_expect_tx(bar(full0 + s), L::kTile);
           armed[s] = int(ph);
           for (int h = 0; h < D / 64; ++h)
@@ -269,16 +273,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     // Issue P_pv V_pv (pv >= 0) interleaved with S_sa, S_sb (>= 0), then
     // signal: S_full / K_empty per S, PV_done / V_empty for the product,
-    // Q_empty after the item's last S (last_s).  One thread does all of it:
-    // the waits are single-thread polls, nothing warp-collective on the path.
+    // Q_empty after the item's last S (last_s).  The whole warp runs the
+    // loop (its control and descriptors stay warp-uniform); one elected lane
+    // issues each MMA and commit.
     auto issue = [&](int64_t pv, bool pv_first, int64_t sa, int64_t sb, int64_t last_s) {
-      if (sa >= 0 && !(ok = wait_bar(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
-      if (sb >= 0 && !(ok = wait_bar(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
+      if (sa >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
+      if (sb >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
       if (pv >= 0) {
-        if (!(ok = wait_bar(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
+        if (!(ok = wait_warp(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
         // P_pv written (and, for a partial paged chunk, the V rows past the
         // used length zeroed by the softmax warps)
-        if (!(ok = wait_bar(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
+        if (!(ok = wait_warp(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
       }
       tc_fence_after();
       const uint32_t pa = tS0 + uint32_t(pv % kSBufs) * 128u;
@@ -289,33 +294,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
         if (pv >= 0)
-          mma_ts(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
+          mma_ts_e(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
         if (kk < D / 16) {
-          if (sa >= 0) mma_ss(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
-          if (sb >= 0) mma_ss(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          if (sa >= 0) mma_ss_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          if (sb >= 0) mma_ss_e(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
         }
       }
-      if (sa >= 0) { mma_commit(bar(kBarSFull + int(sa % kSBufs))); mma_commit(bar(kBarKEmpty + int(sa % kStages))); }
-      if (sb >= 0) { mma_commit(bar(kBarSFull + int(sb % kSBufs))); mma_commit(bar(kBarKEmpty + int(sb % kStages))); }
-      if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit(bar(kBarQEmpty));
-      if (pv >= 0) { mma_commit(bar(kBarPVDone + int(pv & 1))); mma_commit(bar(kBarVEmpty + int(pv % kStages))); }
+      if (sa >= 0) { mma_commit_e(bar(kBarSFull + int(sa % kSBufs))); mma_commit_e(bar(kBarKEmpty + int(sa % kStages))); }
+      if (sb >= 0) { mma_commit_e(bar(kBarSFull + int(sb % kSBufs))); mma_commit_e(bar(kBarKEmpty + int(sb % kStages))); }
+      if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit_e(bar(kBarQEmpty));
+      if (pv >= 0) { mma_commit_e(bar(kBarPVDone + int(pv & 1))); mma_commit_e(bar(kBarVEmpty + int(pv % kStages))); }
     };
-    if (lane == 0) {
-      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const ItemView v = item_view(p, p.fwd_items[it]);
-        const int n = count_chunks(p, v);
-        if (n == 0) continue;
-        if (!(ok = wait_bar(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
-        ++q_it;
-        const int64_t t0 = kv_it, last = kv_it + n - 1;
-        issue(-1, false, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
-        for (int j = 0; j < n && ok; ++j) issue(t0 + j, j == 0, j + 2 < n ? t0 + j + 2 : -1, -1, last);
-        kv_it += uint32_t(n);
-      }
-      if (*abort) {  // let issued MMAs finish before TMEM is freed
-        mma_commit(bar(kBarDrain));
-        drain_wait(bar(kBarDrain), 0);
-      }
+    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+      const ItemView v = item_view(p, p.fwd_items[it]);
+      const int n = count_chunks(p, v);
+      if (n == 0) continue;
+      if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
+      ++q_it;
+      const int64_t t0 = kv_it, last = kv_it + n - 1;
+      issue(-1, false, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
+      for (int j = 0; j < n && ok; ++j) issue(t0 + j, j == 0, j + 2 < n ? t0 + j + 2 : -1, -1, last);
+      kv_it += uint32_t(n);
+    }
+    if (*abort) {  // let issued MMAs finish before TMEM is freed
+      mma_commit_e(bar(kBarDrain));
+      if (lane == 0) drain_wait(bar(kBarDrain), 0);
     }
     __syncwarp();
   } else if (warp < kLoadWarp) {
@@ -361,10 +364,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t tS = tS0 + uint32_t(b) * 128u + lane_off;
           const int valid_all = v.kvlen - v.u0(ch);       // kv columns of the chunk that exist
           const int valid = valid_all - kCols * wg;        // of this group's columns
-          if (p.kv_layout == BSA_LAYOUT_PA_BBND && valid_all < 128) {
-            // rows of the last page past the used length may hold anything
-            // (even NaN); their P is 0, so make their V exactly 0 as well
-            // (before P is published: the MMA reads V after P_full)
+          if (valid_all < 128) {
+            // kv rows past the used length may hold anything (the rest of a
+            // page, another sequence's tokens, even NaN); their P is (nearly)
+            // 0, so make their V exactly 0 as well (before P is published:
+            // the MMA reads V after P_full)
             const int st = int(kv_it % kStages);
             if (!(ok = wait_warp(bar(kBarVFull + st), (kv_it / kStages) & 1u, abort, p.status))) break;
             uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + st * L::kTile);
@@ -383,12 +387,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < kCols; ++c)
               if (c >= valid) x[c] = __float_as_uint(-INFINITY);
           }
+          // P = exp2(scale*log2(e)*s - m) over this group's columns, with the
+          // row sum of this half
+          float ps[2] = {0.f, 0.f};
+          uint32_t pk[kCols / 2];
+          auto exps = [&](float mm) {
+            ps[0] = ps[1] = 0.f;
+#pragma unroll
+            for (int c = 0; c < kCols; c += 2) {
+              const float a0 = fmaf(__uint_as_float(x[c]), p.scale_log2, -mm);
+              const float a1 = fmaf(__uint_as_float(x[c + 1]), p.scale_log2, -mm);
+              const bool poly = ((c >> 1) & 7) < kPolyPairsOf8;  // fixed per unrolled c
+              const float e0 = poly ? exp2_poly(a0) : ex2(a0);
+              const float e1 = poly ? exp2_poly(a1) : ex2(a1);
+              ps[(c >> 1) & 1] += e0 + e1;
+              pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+            }
+          };
+          const bool first = m == -INFINITY;
+          // After the first chunk P is computed at once against the current
+          // reference m; the half-row max only decides whether the row needs
+          // a new reference (rare), in which case P is computed again.
+          if (!first) exps(m);
           float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < kCols; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(x[c]));
           const float hmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
           // does any row of this warp's columns need a new max?
-          const bool first = m == -INFINITY;
           const uint32_t need = __any_sync(0xffffffffu, first || hmax > m + kRescaleThreshold) ? 1u : 0u;
           if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
           if (!rendezvous()) break;
@@ -405,14 +430,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll 1
             for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) {
               if (g2 == wg) continue;
-              uint32_t y[kCols];
-              tmem_ld_cols<kCols>(tS + uint32_t(kCols * g2), y);
-              tmem_wait_ld();
               float ym = -INFINITY;
-              const int vy = valid_all - kCols * g2;
+#pragma unroll 1
+              for (int h = 0; h < 2; ++h) {  // in halves: fewer live registers
+                uint32_t y[kCols / 2];
+                tmem_ld_cols<kCols / 2>(tS + uint32_t(kCols * g2 + (kCols / 2) * h), y);
+                tmem_wait_ld();
+                const int vy = valid_all - kCols * g2 - (kCols / 2) * h;
 #pragma unroll
-              for (int c = 0; c < kCols; ++c)
-                if (c < vy) ym = fmaxf(ym, __uint_as_float(y[c]));
+                for (int c = 0; c < kCols / 2; ++c)
+                  if (c < vy) ym = fmaxf(ym, __uint_as_float(y[c]));
+              }
               cm = fmaxf(cm, ym * p.scale_log2);
             }
             // nobody overwrites S with P before every thread has read it
@@ -420,16 +448,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float m_new = fmaxf(m, cm);
             alpha = first ? 1.f : ex2(m - m_new);
             m = m_new;
-          }
-          // P = exp2(scale*log2(e)*s - m) over this group's columns
-          float ps[2] = {0.f, 0.f};
-          uint32_t pk[kCols / 2];
-#pragma unroll
-          for (int c = 0; c < kCols; c += 2) {
-            const float e0 = ex2(fmaf(__uint_as_float(x[c]), p.scale_log2, -m));
-            const float e1 = ex2(fmaf(__uint_as_float(x[c + 1]), p.scale_log2, -m));
-            ps[(c >> 1) & 1] += e0 + e1;
-            pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+            exps(m);
           }
           // P over the first half of this group's own S columns: no other
           // warp reads them any more (the grow path's reads of the other

@@ -16,23 +16,40 @@ static __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
-// Bounded wait: gives up after kWaitNs of wall time (raising the abort flag
-// and BSA_FLAG_TIMEOUT), or as soon as another role has aborted.
+// Longest single hardware suspension of a waiting thread (ns).  A thread
+// whose barrier never completes (another role aborted) notices the abort flag
+// within this time.
+constexpr uint32_t kSuspendNs = 200000;
+
+// Bounded wait: the thread sleeps in the barrier (no polling loop competing
+// for issue slots with the math warps) and gives up after kWaitNs of wall
+// time (raising the abort flag and BSA_FLAG_TIMEOUT), or as soon as another
+// role has aborted.
 static __device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort,
                                          uint32_t *status) {
   if (sm100::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (sm100::mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0u) {
-      if (*abort) return false;
-      if (global_ns() - t0 > kWaitNs) {
-        *abort = 1;
-        atomicOr(status + kStFlags, BSA_FLAG_TIMEOUT);
-        return false;
-      }
+  for (;;) {
+    if (sm100::mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitNs) {
+      *abort = 1;
+      atomicOr(status + kStFlags, BSA_FLAG_TIMEOUT);
+      return false;
     }
   }
+}
+
+// Producers run ahead of their consumers; the same wait serves them.
+static __device__ __forceinline__ bool wait_bar_lazy(uint32_t bar, uint32_t parity,
+                                              volatile int *abort, uint32_t *status) {
+  return wait_bar(bar, parity, abort, status);
+}
+
+static __device__ __forceinline__ bool wait_warp_lazy(uint32_t bar, uint32_t parity,
+                                               volatile int *abort, uint32_t *status) {
+  const bool r = wait_bar(bar, parity, abort, status);
+  return __all_sync(0xffffffffu, r);
 }
 
 // the same, agreed by the whole warp (tcgen05 .sync.aligned ops follow)

@@ -264,6 +264,15 @@ bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, co
  * workspace passes the pair on to its bsa_fwd. */
 bsa_status bsa_set_main_kernel_events(void *before, void *after);
 
+/* Diagnostic (the pages have no counterpart).  For n floats x (device
+ * memory), writes y_poly[i] = the FMA-pipe 2^x the softmax kernels use for part
+ * of their exponentials (range reduction plus a degree-3 minimax polynomial,
+ * relative error <= 7.5e-5 for x >= -126) and y_mufu[i] = the hardware
+ * ex2.approx of x, asynchronously on `stream`.  Caller-owned device buffers;
+ * BSA_ERR_NULLPTR for a NULL buffer with n > 0, BSA_ERR_PARAM_INVALID for
+ * n < 0, BSA_ERR_CUDA if the launch fails. */
+bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, void *stream);
+
 /* Library ABI version (bumped on any signature or layout change). */
 int32_t bsa_abi_version(void);
 
