@@ -6,9 +6,10 @@
 // head h2; its K and V stay in shared memory and dK, dV accumulate in TMEM
 // while the item walks, for every q head of the GQA group, the query blocks
 // that selected its kv block (the inverted index) in 128-row q steps:
-//   phase 1 (two interleaved MMA chains):
-//     S^T  = K Q^T          -> TMEM R0        (M = kv, N = q, K = D)
-//     dP^T = V dOut^T       -> TMEM R1
+//   phase 1:
+//     S^T  = K Q^T          -> TMEM R0        (M = kv, N = q, K = D), issued
+//                              as soon as the previous step's phase 2 is done
+//     dP^T = V dOut^T       -> TMEM R1        once the previous dQ left R1
 //   softmax warps (thread = kv row, group w = q columns [64w, 64w+64)):
 //     P^T  = exp2(scale*log2(e)*S^T - lse*log2(e))   (0 for rows/cols outside)
 //     dS^T = P^T o (dP^T - Dsum)
@@ -346,18 +347,26 @@ __global__ void __launch_bounds__(kBThreads, 1)
       for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
         const int slot = int(sk & 1u);
         if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
-        // R1 still holds the previous step's dQ until it has been read out
-        if (sk > 0 && !(ok = wait_warp(bar(kBarDQOut + ((sk - 1) & 1u)), ((sk - 1) >> 1) & 1u, abort, p.status)))
-          break;
+        // R0 held the previous step's P and dS until its phase-2 MMAs were
+        // done: S^T may start while the previous dQ is still being read out
+        if (sk > 0 && !(ok = wait_warp(bar(kBarP2), (sk - 1) & 1u, abort, p.status))) break;
         tc_fence_after();
         const uint64_t dQk = sw128_desc(sQ + slot * L::kTile, 16, 1024);
         const uint64_t dOk = sw128_desc(sDO + slot * L::kTile, 16, 1024);
         if (lane == 0) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
+          for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tR0, dKk + kstep(kk), dQk + kstep(kk), idSP, kk > 0 ? 1u : 0u);
+        }
+        __syncwarp();
+        // R1 still holds the previous step's dQ until it has been read out
+        if (sk > 0 && !(ok = wait_warp(bar(kBarDQOut + ((sk - 1) & 1u)), ((sk - 1) >> 1) & 1u, abort, p.status)))
+          break;
+        tc_fence_after();
+        if (lane == 0) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
             mma_ss(tR1, dVk + kstep(kk), dOk + kstep(kk), idSP, kk > 0 ? 1u : 0u);
-          }
           mma_commit(bar(kBarS));
         }
         __syncwarp();
@@ -416,22 +425,32 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const float *lse2 = stat + slot * 256;
         const float *dsum = lse2 + 128;
         uint32_t pp[32], dd[32];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t xs[32], xd[32];
-          const uint32_t col = uint32_t(64 * wg + 32 * h);
-          tmem_ld32(tR0 + lane_off + col, xs);
-          tmem_ld32(tR1 + lane_off + col, xd);
+        {
+          // 16-column blocks of S^T and dP^T, the next block's TMEM loads in
+          // flight while this one is computed
+          const uint32_t c0 = uint32_t(64 * wg);
+          uint32_t xs[2][16], xd[2][16];
+          tmem_ld16(tR0 + lane_off + c0, xs[0]);
+          tmem_ld16(tR1 + lane_off + c0, xd[0]);
           tmem_wait_ld();
 #pragma unroll
-          for (int c2 = 0; c2 < 32; c2 += 2) {
-            const int q = int(col) + c2;
-            const float p0 = kv_ok ? ex2(fmaf(__uint_as_float(xs[c2]), p.scale_log2, -lse2[q])) : 0.f;
-            const float p1 = kv_ok ? ex2(fmaf(__uint_as_float(xs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
-            const float s0 = p0 * (__uint_as_float(xd[c2]) - dsum[q]);
-            const float s1 = p1 * (__uint_as_float(xd[c2 + 1]) - dsum[q + 1]);
-            pp[16 * h + (c2 >> 1)] = MmaOp<T>::pack(p0, p1);
-            dd[16 * h + (c2 >> 1)] = MmaOp<T>::pack(s0, s1);
+          for (int k = 0; k < 4; ++k) {
+            if (k + 1 < 4) {
+              tmem_ld16(tR0 + lane_off + c0 + uint32_t(16 * (k + 1)), xs[(k + 1) & 1]);
+              tmem_ld16(tR1 + lane_off + c0 + uint32_t(16 * (k + 1)), xd[(k + 1) & 1]);
+            }
+            const uint32_t *bs = xs[k & 1], *bd = xd[k & 1];
+#pragma unroll
+            for (int c2 = 0; c2 < 16; c2 += 2) {
+              const int q = int(c0) + 16 * k + c2;
+              const float p0 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2]), p.scale_log2, -lse2[q])) : 0.f;
+              const float p1 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
+              const float s0 = p0 * (__uint_as_float(bd[c2]) - dsum[q]);
+              const float s1 = p1 * (__uint_as_float(bd[c2 + 1]) - dsum[q + 1]);
+              pp[8 * k + (c2 >> 1)] = MmaOp<T>::pack(p0, p1);
+              dd[8 * k + (c2 >> 1)] = MmaOp<T>::pack(s0, s1);
+            }
+            if (k + 1 < 4) tmem_wait_ld();
           }
         }
         // P and dS into this group's own R0 columns (no other group reads
