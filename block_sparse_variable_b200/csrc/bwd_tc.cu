@@ -332,9 +332,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
       if (!(ok = wait_warp(bar(kBarKV), kv_it & 1u, abort, p.status))) break;
       ++kv_it;
       const int valid = v.kvlen - v.u0;
-      if (p.kv_layout == BSA_LAYOUT_PA_BBND && valid < 128) {
-        // rows of the last page past the used length may hold anything
-        // (even NaN): zero them in K and V so that they contribute nothing
+      if (valid < 128) {
+        // kv rows past the used length (the rest of a page, another
+        // sequence's tokens, padding) may hold anything, even NaN: zero them
+        // in K and V so that they contribute nothing (valid >= 1: an item
+        // exists only for a slice that starts below kvlen)
         for (int w = lane; w < (128 - valid) * 8 * (D / 64); w += 32) {
           const int h = w / ((128 - valid) * 8), x = w % ((128 - valid) * 8);
           reinterpret_cast<uint4 *>(sbase + L::kK + h * L::kBox)[valid * 8 + x] = make_uint4(0, 0, 0, 0);

@@ -7,16 +7,14 @@
 //
 // One persistent CTA per SM; each work item is 128 query rows of one head,
 // walked over 128-row kv chunks t of the selected blocks.
-// Warp roles (352 threads):
+// Warp roles (384 threads):
 //   warp 8      TMA: the Q tile once per item, then K chunks (3-stage ring)
 //   warp 10     TMA: the matching V chunks (3-stage ring)
-//   warp 9      TMEM owner and MMA issuer (one elected lane).  It keeps two
-//               independent accumulation chains in flight: the P_t V_t
-//               product (TS form, P read from TMEM) is interleaved MMA by MMA
-//               with S_{t+2} = Q K_{t+2}^T (SS form), since one chain of
-//               dependent MMAs into a single accumulator runs at about half
-//               the tensor rate.  Descriptors are precomputed and advanced
-//               by adding to their address field.
+//   warp 9      TMEM owner; issues O += P_t V_t (TS form, P read from TMEM)
+//   warp 11     issues S_t = Q K_t^T (SS form), up to two chunks ahead of the
+//               softmax.  The MMA issue is split over two schedulers because
+//               an MMA issued into a full tensor-pipe queue stalls in issue and
+//               holds up the softmax warps that share its scheduler.
 //   warps 0..7  two softmax warpgroups; thread (group w, row r) owns kv
 //               columns [64w, 64w+64) of query row r in every chunk.  The
 //               running max m (log2 domain) is kept stale until a row's max
@@ -50,12 +48,13 @@ using namespace sm100;
 
 constexpr int kSoftmaxGroups = 2;  // warpgroups sharing the kv columns of a chunk
 constexpr int kSoftmaxThreads = 128 * kSoftmaxGroups;
-constexpr int kTcThreads = kSoftmaxThreads + 96;  // + Q/K loads, MMA, V loads
+constexpr int kTcThreads = kSoftmaxThreads + 128;  // + Q/K loads, PV MMAs, V loads, S MMAs
 constexpr int kStages = 3;       // depth of the K ring and of the V ring
 constexpr int kSBufs = 3;        // S / P buffers in TMEM
 constexpr int kLoadWarp = 4 * kSoftmaxGroups;
 constexpr int kMmaWarp = kLoadWarp + 1;
 constexpr int kVLoadWarp = kLoadWarp + 2;
+constexpr int kSMmaWarp = kLoadWarp + 3;
 constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
 // of every 8 column pairs, this many take their exponentials on the FMA pipe
@@ -75,8 +74,10 @@ enum : int {
   kBarPVDone = 20,  // + (chunk index & 1): P_t V_t is in O
   kBarXchg = 22,    // + row quarter: rendezvous of the warps that share 32 query
                     // rows (one per group; 32 arrivals per warp)
-  kBarDrain = 26,
-  kNumBars = 27
+  kBarDrain = 26,   // the P V issuer's MMAs on the abort path
+  kBarSFree = 27,   // + S buffer: the P V product that read the buffer's P is done
+  kBarDrainS = 30,  // the S issuer's MMAs on the abort path
+  kNumBars = 31
 };
 
 template <int D>
@@ -193,6 +194,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(bar(kBarPVDone + 1), 1);
     for (int q = 0; q < 4; ++q) mbar_init(bar(kBarXchg + q), kSoftmaxThreads / 4);
     mbar_init(bar(kBarDrain), 1);
+    mbar_init(bar(kBarDrainS), 1);
+    for (int b = 0; b < kSBufs; ++b) mbar_init(bar(kBarSFree + b), 1);
     *abort = 0;
     fence_barrier_init();
   }
@@ -255,8 +258,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (armed[s] >= 0) drain_wait(bar(full0 + s), uint32_t(armed[s]));
       }
     }
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------- MMA issuer
+  } else if (warp == kMmaWarp || warp == kSMmaWarp) {
+    // -------------------------------------------------------- MMA issuers
+    // Two warps on two different schedulers issue the MMAs: an MMA issued
+    // into a full tensor-pipe queue stalls in issue and holds up the softmax
+    // warps that share its scheduler, so the load is split.  S_t = Q K_t^T
+    // (SS form) and O += P_t V_t (TS form, P read from TMEM) are independent
+    // chains; S_t overwrites the buffer of P_{t-3} only after P_{t-3} V_{t-3}
+    // is done (S_free).  Each warp runs its loop warp-uniformly (descriptors
+    // precomputed and advanced by adding to their address field) and one
+    // elected lane issues each MMA and commit.
     constexpr uint32_t idS = idesc_f16(BF16, 128, 128, false, false);
     constexpr uint32_t idPV = idesc_f16(BF16, 128, D, false, true);
     // descriptors: K-major Q / K (a 16-element K step is +32 B, the second
@@ -269,56 +280,57 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // 16 kv columns of P = 8 TMEM columns; the first 64 kv columns' P is in
     // TMEM columns [0, 32), the next 64's in [64, 96) of the S buffer
     auto pcol = [](int kk) { return uint32_t(64 * (kk >> 2) + 8 * (kk & 3)); };
+    const bool is_s = warp == kSMmaWarp;
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
-    // Issue P_pv V_pv (pv >= 0) interleaved with S_sa, S_sb (>= 0), then
-    // signal: S_full / K_empty per S, PV_done / V_empty for the product,
-    // Q_empty after the item's last S (last_s).  The whole warp runs the
-    // loop (its control and descriptors stay warp-uniform); one elected lane
-    // issues each MMA and commit.
-    auto issue = [&](int64_t pv, bool pv_first, int64_t sa, int64_t sb, int64_t last_s) {
-      if (sa >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sa % kStages)), uint32_t(sa / kStages) & 1u, abort, p.status))) return;
-      if (sb >= 0 && !(ok = wait_warp(bar(kBarKFull + int(sb % kStages)), uint32_t(sb / kStages) & 1u, abort, p.status))) return;
-      if (pv >= 0) {
-        if (!(ok = wait_warp(bar(kBarVFull + int(pv % kStages)), uint32_t(pv / kStages) & 1u, abort, p.status))) return;
-        // P_pv written (and, for a partial paged chunk, the V rows past the
-        // used length zeroed by the softmax warps)
-        if (!(ok = wait_warp(bar(kBarPFull + int(pv % kSBufs)), uint32_t(pv / kSBufs) & 1u, abort, p.status))) return;
-      }
-      tc_fence_after();
-      const uint32_t pa = tS0 + uint32_t(pv % kSBufs) * 128u;
-      const uint64_t vd = dV + uint64_t((pv % kStages) * (L::kTile >> 4));
-      const uint32_t da = tS0 + uint32_t(sa % kSBufs) * 128u, db = tS0 + uint32_t(sb % kSBufs) * 128u;
-      const uint64_t ka = dK + uint64_t((sa % kStages) * (L::kTile >> 4));
-      const uint64_t kb = dK + uint64_t((sb % kStages) * (L::kTile >> 4));
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        if (pv >= 0)
-          mma_ts_e(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (pv_first && kk == 0) ? 0u : 1u);
-        if (kk < D / 16) {
-          if (sa >= 0) mma_ss_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
-          if (sb >= 0) mma_ss_e(db, dQ + kstep(kk), kb + kstep(kk), idS, kk > 0 ? 1u : 0u);
-        }
-      }
-      if (sa >= 0) { mma_commit_e(bar(kBarSFull + int(sa % kSBufs))); mma_commit_e(bar(kBarKEmpty + int(sa % kStages))); }
-      if (sb >= 0) { mma_commit_e(bar(kBarSFull + int(sb % kSBufs))); mma_commit_e(bar(kBarKEmpty + int(sb % kStages))); }
-      if (last_s >= 0 && (sa == last_s || sb == last_s)) mma_commit_e(bar(kBarQEmpty));
-      if (pv >= 0) { mma_commit_e(bar(kBarPVDone + int(pv & 1))); mma_commit_e(bar(kBarVEmpty + int(pv % kStages))); }
-    };
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const ItemView v = item_view(p, p.fwd_items[it]);
       const int n = count_chunks(p, v);
       if (n == 0) continue;
-      if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
-      ++q_it;
-      const int64_t t0 = kv_it, last = kv_it + n - 1;
-      issue(-1, false, t0, n > 1 ? t0 + 1 : -1, last);  // S_0 and S_1 together
-      for (int j = 0; j < n && ok; ++j) issue(t0 + j, j == 0, j + 2 < n ? t0 + j + 2 : -1, -1, last);
+      if (is_s) {
+        if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
+        ++q_it;
+        for (int j = 0; j < n && ok; ++j) {
+          const uint32_t t = kv_it + uint32_t(j);
+          const int b = int(t % kSBufs), st = int(t % kStages);
+          if (t >= uint32_t(kSBufs) &&
+              !(ok = wait_warp(bar(kBarSFree + b), (t / kSBufs - 1) & 1u, abort, p.status)))
+            break;
+          if (!(ok = wait_warp(bar(kBarKFull + st), (t / kStages) & 1u, abort, p.status))) break;
+          tc_fence_after();
+          const uint32_t da = tS0 + uint32_t(b) * 128u;
+          const uint64_t ka = dK + uint64_t(st * (L::kTile >> 4));
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) mma_ss_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          mma_commit_e(bar(kBarSFull + b));
+          mma_commit_e(bar(kBarKEmpty + st));
+          if (j == n - 1) mma_commit_e(bar(kBarQEmpty));
+        }
+      } else {
+        for (int j = 0; j < n && ok; ++j) {
+          const uint32_t t = kv_it + uint32_t(j);
+          const int b = int(t % kSBufs), st = int(t % kStages);
+          if (!(ok = wait_warp(bar(kBarVFull + st), (t / kStages) & 1u, abort, p.status))) break;
+          // P_t written (and, for a partial chunk, the V rows past the used
+          // length zeroed by the softmax warps)
+          if (!(ok = wait_warp(bar(kBarPFull + b), (t / kSBufs) & 1u, abort, p.status))) break;
+          tc_fence_after();
+          const uint32_t pa = tS0 + uint32_t(b) * 128u;
+          const uint64_t vd = dV + uint64_t(st * (L::kTile >> 4));
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_ts_e(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (j == 0 && kk == 0) ? 0u : 1u);
+          mma_commit_e(bar(kBarPVDone + int(t & 1u)));
+          mma_commit_e(bar(kBarVEmpty + st));
+          mma_commit_e(bar(kBarSFree + b));
+        }
+      }
       kv_it += uint32_t(n);
     }
     if (*abort) {  // let issued MMAs finish before TMEM is freed
-      mma_commit_e(bar(kBarDrain));
-      if (lane == 0) drain_wait(bar(kBarDrain), 0);
+      const int dr = is_s ? kBarDrainS : kBarDrain;
+      mma_commit_e(bar(dr));
+      if (lane == 0) drain_wait(bar(dr), 0);
     }
     __syncwarp();
   } else if (warp < kLoadWarp) {

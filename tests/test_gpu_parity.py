@@ -154,6 +154,46 @@ def test_edge_cases(name):
     _run_and_check(_problem(name))
 
 
+def _poison_unused_kv(p):
+    """NaN in every stored K/V row the attention must not use: rows past
+    seqused_kv (BNSD, TND), the tail of each last page and whole unused pages
+    (PA_BBND).  Results must not change and must stay finite."""
+    k, v = p.k.clone(), p.v.clone()
+    lens = p.lens_kv
+    if p.layout_kv == "BNSD":
+        for b, n in enumerate(lens):
+            k[b, :, n:] = float("nan")
+            v[b, :, n:] = float("nan")
+    elif p.layout_kv == "TND":
+        cu = p.cu_kv.tolist()
+        for b, n in enumerate(lens):
+            k[cu[b] + n:cu[b + 1]] = float("nan")
+            v[cu[b] + n:cu[b + 1]] = float("nan")
+    else:
+        used = set()
+        ps = p.page_size
+        for b, n in enumerate(lens):
+            for j in range((n + ps - 1) // ps):
+                pg = int(p.block_table[b, j])
+                used.add(pg)
+                if (j + 1) * ps > n:
+                    k[pg, n - j * ps:] = float("nan")
+                    v[pg, n - j * ps:] = float("nan")
+        for pg in range(k.shape[0]):
+            if pg not in used:
+                k[pg] = float("nan")
+                v[pg] = float("nan")
+    p.k, p.v = k, v
+    return p
+
+
+@pytest.mark.parametrize("name", ["bnsd_ragged_kv", "tnd_seqused", "paged", "paged_256"])
+def test_nan_in_unused_kv_rows(name):
+    p = _poison_unused_kv(_problem(name))
+    assert torch.isnan(p.k.float()).any()
+    _run_and_check(p)
+
+
 @pytest.mark.parametrize("c", [1, 2])
 def test_configs_full(c):
     _run_and_check(workloads.make_config(c))
