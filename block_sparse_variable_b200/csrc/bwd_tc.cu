@@ -244,14 +244,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
       if (lane == 0) {
         mbar_expect_tx(bar(kBarKV), 2 * L::kTile);
         armed_kv = int(kv_it & 1u);
-        int c1, c2, c3;
-        if (p.kv_layout == BSA_LAYOUT_PA_BBND) { c1 = v.h2; c2 = v.u0 % p.page_size; c3 = v.pg; }
-        else if (p.kv_layout == BSA_LAYOUT_TND) { c1 = int(v.bi.kv_tok0) + v.u0; c2 = v.h2; c3 = 0; }
-        else { c1 = v.u0; c2 = v.h2; c3 = v.b; }
-        for (int h = 0; h < D / 64; ++h) {
-          tma_load_4d(sK + h * L::kBox, &map_k, bar(kBarKV), h * 64, c1, c2, c3);
-          tma_load_4d(sV + h * L::kBox, &map_v, bar(kBarKV), h * 64, c1, c2, c3);
-        }
+        int row, last;  // tile coordinates: (0, row, 0, h2, last)
+        if (p.kv_layout == BSA_LAYOUT_PA_BBND) { row = v.u0 % p.page_size; last = v.pg; }
+        else if (p.kv_layout == BSA_LAYOUT_TND) { row = int(v.bi.kv_tok0) + v.u0; last = 0; }
+        else { row = v.u0; last = v.b; }
+        tma_load_5d(sK, &map_k, bar(kBarKV), 0, row, 0, v.h2, last);
+        tma_load_5d(sV, &map_v, bar(kBarKV), 0, row, 0, v.h2, last);
       }
       ++kv_it;
       for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
@@ -293,11 +291,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
           if (refill) bulk_wait_read<1>();
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sQ + slot * L::kTile + h * L::kBox, &map_q, bar(kBarQD + slot), h * 64, tok, h1, bb);
+          tma_load_5d(sQ + slot * L::kTile, &map_q, bar(kBarQD + slot), 0, tok, 0, h1, bb);
           if (refill) bulk_wait_read<0>();
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sDO + slot * L::kTile + h * L::kBox, &map_do, bar(kBarQD + slot), h * 64, tok, h1, bb);
+          tma_load_5d(sDO + slot * L::kTile, &map_do, bar(kBarQD + slot), 0, tok, 0, h1, bb);
         }
         __syncwarp();
         pend_h[slot] = h1;

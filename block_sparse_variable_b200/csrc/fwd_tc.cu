@@ -230,8 +230,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           armed_q = int(q_it & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + v.t0 : v.t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(sQ + h * L::kBox, &map_q, bar(kBarQFull), h * 64, tok, v.h1, bb);
+          tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, 0, v.h1, bb);
           ++q_it;
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) {
@@ -240,15 +239,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int u0 = v.u0(ch);
           int pg;
           page_ok(p, v, u0, pg);
-          int c1, c2, c3;  // coordinates after the head-dim one
-          if (p.kv_layout == BSA_LAYOUT_PA_BBND) { c1 = v.h2; c2 = u0 % p.page_size; c3 = pg; }
-          else if (p.kv_layout == BSA_LAYOUT_TND) { c1 = int(v.bi.kv_tok0) + u0; c2 = v.h2; c3 = 0; }
-          else { c1 = u0; c2 = v.h2; c3 = v.b; }
+          int row, last;  // tile coordinates: (0, row, 0, h2, last)
+          if (p.kv_layout == BSA_LAYOUT_PA_BBND) { row = u0 % p.page_size; last = pg; }
+          else if (p.kv_layout == BSA_LAYOUT_TND) { row = int(v.bi.kv_tok0) + u0; last = 0; }
+          else { row = u0; last = v.b; }
           if (!(ok = wait_bar_lazy(bar(empty0 + s), ph ^ 1u, abort, p.status))) break;
           mbar_expect_tx(bar(full0 + s), L::kTile);
           armed[s] = int(ph);
-          for (int h = 0; h < D / 64; ++h)
-            tma_load_4d(ring + s * L::kTile + h * L::kBox, map, bar(full0 + s), h * 64, c1, c2, c3);
+          tma_load_5d(ring + s * L::kTile, map, bar(full0 + s), 0, row, 0, v.h2, last);
           ++kv_it;
         }
       }

@@ -8,9 +8,12 @@
 
 namespace bsa {
 
-// 128-byte-swizzled 64-column x 128-row boxes of the q / k / v tensors.
-//   q, BNSD/TND kv:  4-D {D, token rows, heads, batch}
-//   PA_BBND kv:      4-D {D, heads, page rows, pages}   (box 64 x 1 x 128 x 1)
+// Whole 128-row tiles of the q / k / v tensors in one copy: 5-D maps
+// {64 columns, rows, D/64 column halves, heads, batch or page} with box
+// {64, 128, D/64, 1, 1}, landing as D/64 consecutive 128-byte-swizzled
+// 128-row x 64-column boxes.  Coordinates (0, row, 0, head, batch/page):
+//   q, BNSD/TND kv:  rows = token rows (TND: batch coordinate 0)
+//   PA_BBND kv:      rows = rows of the page, last coordinate = the page
 struct FwdMaps {
   CUtensorMap q, k, v;
 };
