@@ -57,6 +57,7 @@ constexpr int kVLoadWarp = kLoadWarp + 2;
 constexpr int kSMmaWarp = kLoadWarp + 3;
 constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
 constexpr float kRescaleThreshold = 8.0f;    // log2 units
+constexpr float kRescaleSum = 256.0f;        // 2^kRescaleThreshold
 // of every 8 column pairs, this many take their exponentials on the FMA pipe
 // (exp2_poly) instead of the MUFU unit, which alone would bound the softmax
 constexpr int kPolyPairsOf8 = 0;
@@ -419,12 +420,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // reference m; the half-row max only decides whether the row needs
           // a new reference (rare), in which case P is computed again.
           if (!first) exps(m);
-          float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          auto half_max = [&]() {
+            float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-          for (int c = 0; c < kCols; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(x[c]));
-          const float hmax = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
-          // does any row of this warp's columns need a new max?
-          const uint32_t need = __any_sync(0xffffffffu, first || hmax > m + kRescaleThreshold) ? 1u : 0u;
+            for (int c = 0; c < kCols; ++c) pm[c & 3] = fmaxf(pm[c & 3], __uint_as_float(x[c]));
+            return fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3])) * p.scale_log2;
+          };
+          // does any row of this warp's columns need a new reference?  After
+          // the first chunk the half-row sum of P decides: below 2^8 every P
+          // is below 2^8 (a larger sum may call for a new reference that turns
+          // out to change little, which is still exact); no max is needed.
+          const uint32_t need =
+              __any_sync(0xffffffffu, first || !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
           if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
           if (!rendezvous()) break;
           // one decision for the rows of this warp, shared with the other
@@ -436,7 +443,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const bool grow = any != 0u;
           if (grow) {
             // the full row max: the other groups' columns are still S in TMEM
-            float cm = hmax;
+            float cm = half_max();
 #pragma unroll 1
             for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) {
               if (g2 == wg) continue;
