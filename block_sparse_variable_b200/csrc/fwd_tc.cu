@@ -56,8 +56,9 @@ constexpr int kMmaWarp = kLoadWarp + 1;
 constexpr int kVLoadWarp = kLoadWarp + 2;
 constexpr int kSMmaWarp = kLoadWarp + 3;
 constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
-constexpr float kRescaleThreshold = 8.0f;    // log2 units
-constexpr float kRescaleSum = 256.0f;        // 2^kRescaleThreshold
+// a row takes a new reference max once its P could exceed 2^8 (a half-row
+// sum of P above 2^8)
+constexpr float kRescaleSum = 256.0f;
 // of every 8 column pairs, this many take their exponentials on the FMA pipe
 // (exp2_poly) instead of the MUFU unit, which alone would bound the softmax
 constexpr int kPolyPairsOf8 = 0;
@@ -233,6 +234,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
           tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, 0, v.h1, bb);
           ++q_it;
+          // the next item's Q tile into L2 now: its load waits for this
+          // item's last S, and a miss to memory then would stall the pipeline
+          if (it + int(gridDim.x) < n_items) {
+            const ItemView w = item_view(p, p.fwd_items[it + gridDim.x]);
+            tma_prefetch_l2_5d(&map_q, 0, p.q_layout == BSA_LAYOUT_TND ? int(w.bi.q_tok0) + w.t0 : w.t0, 0,
+                               w.h1, p.q_layout == BSA_LAYOUT_TND ? 0 : w.b);
+          }
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) {
           const int s = int(kv_it % kStages);
@@ -513,19 +521,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       constexpr int kOc = D / kSoftmaxGroups;  // output columns per group
       if (n > 0) {
 #pragma unroll
-        for (int q = 0; q < kOc / 16; ++q) {
-          const uint32_t col = uint32_t(wg * kOc + q * 16);
-          uint32_t o[16];
-          tmem_ld16(tO + lane_off + col, o);
+        for (int q = 0; q < kOc / 32; ++q) {
+          const uint32_t col = uint32_t(wg * kOc + q * 32);
+          uint32_t o[32];
+          tmem_ld32(tO + lane_off + col, o);
           tmem_wait_ld();
           if (live) {
-            uint4 w[2];
-            uint32_t *wp = reinterpret_cast<uint32_t *>(w);
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-              wp[c] = MmaOp<T>::pack(__uint_as_float(o[2 * c]) * inv, __uint_as_float(o[2 * c + 1]) * inv);
-            reinterpret_cast<uint4 *>(orow + col)[0] = w[0];
-            reinterpret_cast<uint4 *>(orow + col)[1] = w[1];
+            for (int c8 = 0; c8 < 4; ++c8) {
+              uint4 w;
+              w.x = MmaOp<T>::pack(__uint_as_float(o[8 * c8]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
+              w.y = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
+              w.z = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
+              w.w = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
+              reinterpret_cast<uint4 *>(orow + col)[c8] = w;
+            }
           }
         }
       } else if (live) {
