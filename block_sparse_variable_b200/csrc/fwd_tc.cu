@@ -131,11 +131,25 @@ __device__ __forceinline__ Chunk next_chunk(const Problem &p, const ItemView &v,
   if (ch.c >= v.ksl || v.u0(ch) >= v.kvlen) { ++ch.x; ch.c = 0; }
   return settle(p, v, ch);
 }
-__device__ __forceinline__ int count_chunks(const Problem &p, const ItemView &v) {
+// The chunk count of an item, by a whole (converged) warp: each lane takes
+// index entries lane, lane + 32, ... so their loads are in flight together,
+// then the counts are summed.
+__device__ __forceinline__ int count_chunks_warp(const Problem &p, const ItemView &v, int lane) {
   int n = 0;
-  for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) ++n;
+  for (int x = lane; x < v.ncnt; x += 32) {
+    const int base = int(v.crow[x]) * v.BKV;
+    for (int c = 0; c < v.ksl; ++c) {
+      const int u0 = base + c * 128;
+      if (u0 >= v.kvlen) break;
+      int pg;
+      if (page_ok(p, v, u0, pg)) ++n;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
   return n;
 }
+
 
 __device__ __forceinline__ ItemView item_view(const Problem &p, int id) {
   ItemView v;
@@ -225,7 +239,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
         const ItemView v = item_view(p, p.fwd_items[it]);
-        if (count_chunks(p, v) == 0) continue;
+        if (settle(p, v, Chunk{0, 0}).x >= v.ncnt) continue;  // no chunk: nothing to load
         if (is_k) {
           if (!(ok = wait_bar_lazy(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status))) break;
           mbar_expect_tx(bar(kBarQFull), L::kTile);
@@ -234,13 +248,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
           tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, 0, v.h1, bb);
           ++q_it;
-          // the next item's Q tile into L2 now: its load waits for this
-          // item's last S, and a miss to memory then would stall the pipeline
-          if (it + int(gridDim.x) < n_items) {
-            const ItemView w = item_view(p, p.fwd_items[it + gridDim.x]);
-            tma_prefetch_l2_5d(&map_q, 0, p.q_layout == BSA_LAYOUT_TND ? int(w.bi.q_tok0) + w.t0 : w.t0, 0,
-                               w.h1, p.q_layout == BSA_LAYOUT_TND ? 0 : w.b);
-          }
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) {
           const int s = int(kv_it % kStages);
@@ -256,6 +263,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_expect_tx(bar(full0 + s), L::kTile);
           armed[s] = int(ph);
           tma_load_5d(ring + s * L::kTile, map, bar(full0 + s), 0, row, 0, v.h2, last);
+          if (is_k && ch.x == v.ncnt - 1 && ch.c == 0 && it + int(gridDim.x) < n_items) {
+            // the next item's Q tile into L2 as this item's last index entry
+            // starts: its load waits for this item's last S, and a miss to
+            // memory then would stall the pipeline
+            const ItemView w = item_view(p, p.fwd_items[it + gridDim.x]);
+            tma_prefetch_l2_5d(&map_q, 0, p.q_layout == BSA_LAYOUT_TND ? int(w.bi.q_tok0) + w.t0 : w.t0, 0,
+                               w.h1, p.q_layout == BSA_LAYOUT_TND ? 0 : w.b);
+          }
           ++kv_it;
         }
       }
@@ -292,7 +307,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const ItemView v = item_view(p, p.fwd_items[it]);
-      const int n = count_chunks(p, v);
+      const int n = count_chunks_warp(p, v, lane);
       if (n == 0) continue;
       if (is_s) {
         if (!(ok = wait_warp(bar(kBarQFull), q_it & 1u, abort, p.status))) break;
