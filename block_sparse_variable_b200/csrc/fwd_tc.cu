@@ -91,8 +91,8 @@ struct Layout {
   static constexpr int kV = kK + kStages * kTile;
   static constexpr int kBars = kV + kStages * kTile;
   static constexpr int kFlags = kBars + kNumBars * 8;                 // [2][softmax warps] u32
-  static constexpr int kXsum = kFlags + 2 * 4 * kSoftmaxGroups * 4;   // [groups][128] sums
-  static constexpr int kTmemPtr = kXsum + kSoftmaxGroups * 128 * 4;
+  static constexpr int kXsum = kFlags + 2 * 4 * kSoftmaxGroups * 4;   // [2][groups][128] sums
+  static constexpr int kTmemPtr = kXsum + 2 * kSoftmaxGroups * 128 * 4;
   static constexpr int kAbort = kTmemPtr + 4;
   static constexpr int kBytes = kAbort + 4;
   // the dynamic shared window starts 1024-byte aligned (checked at run time)
@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     float *xsum = reinterpret_cast<float *>(sbase + L::kXsum);
     const float kLn2 = 0.6931471805599453f;
     constexpr int kWarps = 4 * kSoftmaxGroups;
-    uint32_t kv_it = 0, x_it = 0;  // global chunk counter; rendezvous counter
+    uint32_t kv_it = 0, x_it = 0, item_n = 0;  // chunk counter; rendezvous counter; items done
     bool ok = true;
     // the warps holding the same 32 query rows (one per group) meet here
     // (bounded: an aborted peer cannot strand us)
@@ -453,15 +453,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // the first chunk the half-row sum of P decides: below 2^8 every P
           // is below 2^8 (a larger sum may call for a new reference that turns
           // out to change little, which is still exact); no max is needed.
-          const uint32_t need =
-              __any_sync(0xffffffffu, first || !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
-          if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
-          if (!rendezvous()) break;
-          // one decision for the rows of this warp, shared with the other
-          // group's warp on the same rows, so that both take the same path
-          uint32_t any = 0;
+          // (the first chunk of an item always takes a reference: both groups
+          // know that without exchanging flags)
+          uint32_t any = 1;
+          if (!first) {
+            const uint32_t need = __any_sync(0xffffffffu, !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
+            if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
+            if (!rendezvous()) break;
+            // one decision for the rows of this warp, shared with the other
+            // group's warp on the same rows, so that both take the same path
+            any = 0;
 #pragma unroll
-          for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) any |= flags[(kv_it & 1u) * kWarps + 4 * g2 + (warp & 3)];
+            for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) any |= flags[(kv_it & 1u) * kWarps + 4 * g2 + (warp & 3)];
+          }
           float alpha = 1.f;
           const bool grow = any != 0u;
           if (grow) {
@@ -524,33 +528,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!(ok = wait_warp(bar(kBarPVDone + int(t & 1u)), (t / 2) & 1u, abort, p.status))) break;
         tc_fence_after();
       }
-      xsum[wg * 128 + r] = l;
+      constexpr int kOc = D / kSoftmaxGroups;  // output columns per group
+      // the row sums of the groups, through slots alternating by item (the
+      // partner reads this item's slot before it can write the slot again)
+      float *xs = xsum + (item_n & 1u) * (kSoftmaxGroups * 128);
+      xs[wg * 128 + r] = l;
       if (!rendezvous()) break;
       float Lsum = 0.f;
 #pragma unroll
-      for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) Lsum += xsum[g2 * 128 + r];
+      for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) Lsum += xs[g2 * 128 + r];
       if (wg == 0 && live && p.lse)
         p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1, v.t0 + r)] =
             Lsum > 0.f ? (m + __log2f(Lsum)) * kLn2 : -INFINITY;
       const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-      constexpr int kOc = D / kSoftmaxGroups;  // output columns per group
       if (n > 0) {
+        uint32_t o[kOc];
+        tmem_ld_cols<kOc>(tO + lane_off + uint32_t(wg * kOc), o);
+        tmem_wait_ld();
+        if (live) {
 #pragma unroll
-        for (int q = 0; q < kOc / 32; ++q) {
-          const uint32_t col = uint32_t(wg * kOc + q * 32);
-          uint32_t o[32];
-          tmem_ld32(tO + lane_off + col, o);
-          tmem_wait_ld();
-          if (live) {
-#pragma unroll
-            for (int c8 = 0; c8 < 4; ++c8) {
-              uint4 w;
-              w.x = MmaOp<T>::pack(__uint_as_float(o[8 * c8]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
-              w.y = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
-              w.z = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
-              w.w = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
-              reinterpret_cast<uint4 *>(orow + col)[c8] = w;
-            }
+          for (int c8 = 0; c8 < kOc / 8; ++c8) {
+            uint4 w;
+            w.x = MmaOp<T>::pack(__uint_as_float(o[8 * c8]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
+            w.y = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
+            w.z = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
+            w.w = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
+            reinterpret_cast<uint4 *>(orow + wg * kOc)[c8] = w;
           }
         }
       } else if (live) {
@@ -558,9 +561,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int c = 0; c < kOc / 8; ++c)
           reinterpret_cast<uint4 *>(orow + wg * kOc)[c] = make_uint4(0, 0, 0, 0);
       }
+      // O is free once every softmax thread has arrived on the next item's
+      // first P_full (the P V issuer waits for it), so no rendezvous here
       tc_fence_before();
-      // every group is done with O and the exchange slots before the next item
-      if (!rendezvous()) break;
+      ++item_n;
     }
   }
   tc_fence_before();
