@@ -82,9 +82,10 @@ def _load():
     lib.bsa_abi_version.restype = ctypes.c_int32
     lib.bsa_set_main_kernel_events.argtypes = [vp, vp]
     lib.bsa_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
+    lib.bsa_selftest_wait_timeout.argtypes = [vp, vp]
     for f in ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_fwd_workspace_layout",
               "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status",
-              "bsa_set_main_kernel_events", "bsa_selftest_exp2"):
+              "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -94,7 +95,7 @@ _lib = _load()
 EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bwd",
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
             "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace",
-            "bsa_set_main_kernel_events", "bsa_selftest_exp2")
+            "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout")
 
 
 def lib():
@@ -311,6 +312,14 @@ def bsa_selftest_exp2(x: torch.Tensor, stream=None):
                                   ctypes.c_void_p(ym.data_ptr()), x.numel(),
                                   ctypes.c_void_p(_stream(stream))), "bsa_selftest_exp2")
     return yp, ym
+
+
+def bsa_selftest_wait_timeout(flags: torch.Tensor, stream=None):
+    """Run the bounded-wait self test; `flags` is a zeroed int32 CUDA tensor
+    whose word 0 receives BSA_FLAG_TIMEOUT."""
+    _check(_lib.bsa_selftest_wait_timeout(ctypes.c_void_p(flags.data_ptr()),
+                                          ctypes.c_void_p(_stream(stream))),
+           "bsa_selftest_wait_timeout")
 
 
 def bsa_set_main_kernel_events(before=None, after=None):

@@ -5,6 +5,7 @@
 #include "bsa_internal.h"
 #include "exp2_poly.cuh"
 #include "ptx_sm80.cuh"
+#include "tc_device.cuh"
 
 namespace bsa {
 namespace {
@@ -18,8 +19,32 @@ __global__ void k_exp2_pair(const float *x, float *y_poly, float *y_mufu, int64_
   }
 }
 
+// One warp waits on an mbarrier that nothing ever arrives at, through the
+// same bounded wait the attention kernels use: the wait must give up after
+// its time limit, raise BSA_FLAG_TIMEOUT in flags[0] and return, leaving the
+// context usable.  Bit 31 would mean the wait wrongly succeeded.
+__global__ void k_wait_timeout(uint32_t *flags) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(b, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = wait_warp(b, 0, &abort_flag, flags);
+  if (threadIdx.x == 0 && ok) atomicOr(flags + kStFlags, 0x80000000u);
+}
+
 }  // namespace
 }  // namespace bsa
+
+extern "C" bsa_status bsa_selftest_wait_timeout(uint32_t *flags, void *stream) {
+  if (!flags) return BSA_ERR_NULLPTR;
+  bsa::k_wait_timeout<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(flags);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
 
 extern "C" bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n,
                                         void *stream) {

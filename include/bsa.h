@@ -273,6 +273,14 @@ bsa_status bsa_set_main_kernel_events(void *before, void *after);
  * n < 0, BSA_ERR_CUDA if the launch fails. */
 bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, void *stream);
 
+/* Diagnostic (the pages have no counterpart).  Launches one warp that waits
+ * on a device barrier nothing ever completes, through the bounded wait every
+ * kernel of this library uses: after its time limit (about 2 s) the wait
+ * gives up, sets BSA_FLAG_TIMEOUT in flags[0] (a caller-owned device word,
+ * zeroed by the caller) and the kernel returns, leaving the context usable.
+ * Asynchronous on `stream`; BSA_ERR_NULLPTR for a NULL flags pointer. */
+bsa_status bsa_selftest_wait_timeout(uint32_t *flags, void *stream);
+
 /* Library ABI version (bumped on any signature or layout change). */
 int32_t bsa_abi_version(void);
 
