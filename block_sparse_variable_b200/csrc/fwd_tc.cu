@@ -8,19 +8,23 @@
 // One persistent CTA per SM; each work item is 128 query rows of one head,
 // walked over 128-row kv chunks t of the selected blocks.
 // Warp roles (384 threads):
-//   warp 8      TMA: the Q tile once per item, then K chunks (3-stage ring)
-//   warp 10     TMA: the matching V chunks (3-stage ring)
+//   warp 8      TMA: the Q tile once per item, then K chunks (3-stage ring);
+//               as an item's last index entry starts, the next item's Q tile
+//               is prefetched into L2
+//   warp 10     TMA: the matching V chunks (3-stage ring); every tile is one
+//               5-D copy of both 64-column halves
 //   warp 9      TMEM owner; issues O += P_t V_t (TS form, P read from TMEM)
 //   warp 11     issues S_t = Q K_t^T (SS form), up to two chunks ahead of the
 //               softmax.  The MMA issue is split over two schedulers because
 //               an MMA issued into a full tensor-pipe queue stalls in issue and
 //               holds up the softmax warps that share its scheduler.
 //   warps 0..7  two softmax warpgroups; thread (group w, row r) owns kv
-//               columns [64w, 64w+64) of query row r in every chunk.  The
-//               running max m (log2 domain) is kept stale until a row's max
-//               grows by more than 2^8 (P stays below 256); only then are the
-//               two halves' maxima exchanged, O and the partial sums l
-//               rescaled.  P = exp2(s*scale*log2 e - m) overwrites S as
+//               columns [64w, 64w+64) of query row r in every chunk.
+//               P = exp2(s*scale*log2 e - m) is computed at once against the
+//               current reference m (log2 domain); only when a half-row sum
+//               of P exceeds 2^8 do the two warps on those rows exchange their
+//               maxima, take a new m, recompute P and rescale O and the
+//               partial sums l.  P overwrites the group's own S columns as
 //               16-bit pairs.  Epilogue: out = O / (l_0 + l_1),
 //               lse = (m + log2(l_0 + l_1)) ln 2.
 // TMEM columns: three S/P buffers [0,128), [128,256), [256,384); O [384,384+D).
