@@ -46,7 +46,8 @@ class _Problem(ctypes.Structure):
                 ("R", ctypes.c_int64), ("W", ctypes.c_int64), ("scale", ctypes.c_double),
                 ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("index", ctypes.c_void_p), ("cu_q", ctypes.c_void_p), ("cu_kv", ctypes.c_void_p),
-                ("seqused_kv", ctypes.c_void_p), ("block_table", ctypes.c_void_p)]
+                ("seqused_kv", ctypes.c_void_p), ("block_table", ctypes.c_void_p),
+                ("causal", ctypes.c_int32)]
 
 
 _lib = None
@@ -104,6 +105,7 @@ class Oracle:
         s.q, s.k, s.v, s.index = (K[n].ctypes.data for n in ("q", "k", "v", "index"))
         s.cu_q, s.cu_kv = _ptr(K["cu_q"]), _ptr(K["cu_kv"])
         s.seqused_kv, s.block_table = _ptr(K["seqused_kv"]), _ptr(K["block_table"])
+        s.causal = int(bool(getattr(p, "causal", False)))
         self._s = s
         self.lib = _load()
 

@@ -19,6 +19,9 @@
  *     lse_t  = m + ln sum_{u in J} exp(s_u - m),   m = max_{u in J} s_u
  *     out_t  = sum_{u in J} exp(s_u - lse_t) * v[u]
  *     J empty -> out_t = 0, lse_t = -inf.
+ *   With the causal mask (GenericBlockSparseAttention, "mask" section: the
+ *   built-in causal mode; aligned to the end of the kv sequence, our
+ *   reading), J(t) also drops every u > t + kvlen_b - qlen_b.
  *
  *   Backward (BlockSparseAttentionGrad README, "Formula"), with out and lse
  *   taken as given inputs:
@@ -66,6 +69,7 @@ typedef struct {
   const int64_t *cu_q, *cu_kv; /* [B+1] or NULL */
   const int32_t *seqused_kv;   /* [B] or NULL */
   const int32_t *block_table;  /* [B, max_pages] or NULL */
+  int32_t causal;              /* 1: u <= t + kvlen_b - qlen_b only */
 } oracle_problem;
 
 /* ---------------------------------------------------------------- lengths */
@@ -153,6 +157,14 @@ static int64_t row_blocks(const oracle_problem *P, int64_t b, int64_t hi, int64_
   return n;
 }
 
+/* One past the last kv token query row t of batch b may see (causal), or
+ * kvlen without the mask. */
+static int64_t visible_end(const oracle_problem *P, int64_t t, int64_t kvlen, int64_t qlen) {
+  if (!P->causal) return kvlen;
+  int64_t e = t + kvlen - qlen + 1;
+  return e < 0 ? 0 : (e < kvlen ? e : kvlen);
+}
+
 static double dot(const double *a, const double *b, int64_t D) {
   double s = 0.0;
   for (int64_t d = 0; d < D; ++d) s += a[d] * b[d];
@@ -174,6 +186,7 @@ int oracle_fwd_rows(const oracle_problem *P, const int64_t *rows, int64_t nrows,
     int64_t nk = ceil_div(kvlen, P->BKV);
     int64_t *blk = (int64_t *)malloc(sizeof(int64_t) * (P->W + 1));
     int64_t nb = row_blocks(P, b, index_head(P, h1), i, qblock_offset(P, b), nk, blk, &f);
+    const int64_t uend = visible_end(P, t, kvlen, q_len(P, b, &f));
     const double *qt = q_row(P, P->q, b, h1, t);
     double *o = out_rows + r * D;
     for (int64_t d = 0; d < D; ++d) o[d] = 0.0;
@@ -182,7 +195,7 @@ int oracle_fwd_rows(const oracle_problem *P, const int64_t *rows, int64_t nrows,
     double m = -INFINITY;
     int64_t count = 0;
     for (int64_t x = 0; x < nb; ++x) {
-      int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < kvlen ? u0 + P->BKV : kvlen;
+      int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < uend ? u0 + P->BKV : uend;
       for (int64_t u = u0; u < u1; ++u) {
         int64_t off = kv_row_offset(P, b, h2, u);
         if (off < 0) { f |= ORACLE_BAD_PAGE; continue; }
@@ -197,7 +210,7 @@ int oracle_fwd_rows(const oracle_problem *P, const int64_t *rows, int64_t nrows,
       /* pass 2: the sum of exponentials and the log-sum-exp */
       double l = 0.0;
       for (int64_t x = 0; x < nb; ++x) {
-        int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < kvlen ? u0 + P->BKV : kvlen;
+        int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < uend ? u0 + P->BKV : uend;
         for (int64_t u = u0; u < u1; ++u) {
           int64_t off = kv_row_offset(P, b, h2, u);
           if (off < 0) continue;
@@ -208,7 +221,7 @@ int oracle_fwd_rows(const oracle_problem *P, const int64_t *rows, int64_t nrows,
       lse_rows[r] = lse;
       /* pass 3: out = sum_u softmax_u * v_u */
       for (int64_t x = 0; x < nb; ++x) {
-        int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < kvlen ? u0 + P->BKV : kvlen;
+        int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < uend ? u0 + P->BKV : uend;
         for (int64_t u = u0; u < u1; ++u) {
           int64_t off = kv_row_offset(P, b, h2, u);
           if (off < 0) continue;
@@ -244,12 +257,13 @@ int oracle_bwd_dq_rows(const oracle_problem *P, const double *out, const double 
     const double *qt = q_row(P, P->q, b, h1, t);
     const double *dOt = q_row(P, dout, b, h1, t);
     const double *ot = q_row(P, out, b, h1, t);
+    const int64_t uend = visible_end(P, t, kvlen, q_len(P, b, &f));
     double lt = lse[row_stat_offset(P, b, h1, t)];
     double sg = dot(dOt, ot, D); /* softmax_grad_t */
     double *dq = dq_rows + r * D;
     for (int64_t d = 0; d < D; ++d) dq[d] = 0.0;
     for (int64_t x = 0; x < nb; ++x) {
-      int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < kvlen ? u0 + P->BKV : kvlen;
+      int64_t u0 = blk[x] * P->BKV, u1 = u0 + P->BKV < uend ? u0 + P->BKV : uend;
       for (int64_t u = u0; u < u1; ++u) {
         int64_t off = kv_row_offset(P, b, h2, u);
         if (off < 0) { f |= ORACLE_BAD_PAGE; continue; }
@@ -293,6 +307,7 @@ int oracle_bwd_dkv_rows(const oracle_problem *P, const double *out, const double
           if (!selected) continue;
           int64_t t1 = (i + 1) * P->BQ < qlen ? (i + 1) * P->BQ : qlen;
           for (int64_t t = i * P->BQ; t < t1; ++t) {
+            if (u >= visible_end(P, t, kvlen, qlen)) continue;
             const double *qt = q_row(P, P->q, b, h1, t);
             const double *dOt = q_row(P, dout, b, h1, t);
             const double *ot = q_row(P, out, b, h1, t);

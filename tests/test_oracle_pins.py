@@ -12,8 +12,8 @@ import torch
 
 import oracle
 import workloads
-from workloads.gen import (make_problem, pat_dense, pat_density, pat_fraction_diag, pat_random_k,
-                           pat_topk)
+from workloads.gen import (make_problem, pat_causal, pat_dense, pat_density, pat_fraction_diag,
+                           pat_random_k, pat_topk)
 from tests import torch_reference as tr
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -285,3 +285,114 @@ def test_config_rows_match_reference(c):
     assert fl == 0
     assert np.allclose(out, o.gather_q(rout, rows).numpy(), atol=1e-11)
     assert np.allclose(lse, o.gather_q(rlse, rows).numpy(), atol=1e-11)
+
+
+# ------------------------------------------------------------ causal mask
+def test_causal_dense_is_sdpa_causal():
+    """Dense index + causal mask == torch scaled_dot_product_attention with
+    is_causal=True (fp64), forward and, through autograd, backward."""
+    p = make_problem(B=1, N1=2, N2=2, D=32, Sq=200, BQ=64, BKV=64, pattern=pat_dense, seed_base=17,
+                     causal=True)
+    o = oracle.Oracle(p)
+    out, lse, fl = o.fwd()
+    assert fl == 0
+    q, k, v = (t.double().requires_grad_() for t in (p.q, p.k, p.v))
+    ref = torch.nn.functional.scaled_dot_product_attention(q, k, v, scale=p.scale, is_causal=True)
+    assert torch.allclose(out, ref.detach(), atol=1e-12, rtol=0)
+    dq, dk, dv, _ = o.bwd(out, p.dout, lse)
+    ref.backward(p.dout.double())
+    for a, r in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        assert torch.allclose(a, r, atol=1e-10, rtol=0), (a - r).abs().max()
+
+
+def test_causal_short_query_is_the_tail_of_a_square_problem():
+    """With fewer query than kv tokens the mask is aligned to the end of the
+    kv sequence: the result equals the last rows of the square causal problem
+    whose last query rows are these."""
+    n_kv, n_q = 150, 40
+    sq = make_problem(layout_q="TND", layout_kv="TND", B=1, N1=2, N2=1, D=16, BQ=32, BKV=32,
+                      lens_q=[n_kv], lens_kv=[n_kv], pattern=pat_dense, seed_base=23, causal=True,
+                      dtype=torch.float64)
+    short = make_problem(layout_q="TND", layout_kv="TND", B=1, N1=2, N2=1, D=16, BQ=32, BKV=32,
+                         lens_q=[n_q], lens_kv=[n_kv], pattern=pat_dense, seed_base=23, causal=True,
+                         dtype=torch.float64)
+    short.q = sq.q[n_kv - n_q:].clone()
+    short.k, short.v = sq.k, sq.v
+    out_sq, lse_sq, _ = oracle.Oracle(sq).fwd()
+    out_sh, lse_sh, fl = oracle.Oracle(short).fwd()
+    assert fl == 0
+    assert torch.allclose(out_sh, out_sq[n_kv - n_q:], atol=1e-13, rtol=0)
+    assert torch.allclose(lse_sh, lse_sq[n_kv - n_q:], atol=1e-13, rtol=0)
+
+
+CAUSAL_CASES = {
+    "bnsd_causal_sparse": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=1, D=32, Sq=300,
+                               pattern=pat_random_k),
+    "tnd_causal_short_q": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=2, D=32,
+                               lens_q=[70, 200], lens_kv=[260, 200], pattern=pat_causal),
+    "paged_causal": dict(layout_q="TND", layout_kv="PA_BBND", B=2, N1=2, N2=1, D=32,
+                         lens_q=[300, 90], lens_kv=[300, 129], page_size=128, pattern=pat_random_k),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CAUSAL_CASES))
+def test_causal_sparse_equals_masked_dense(name):
+    """Sparse + causal == dense attention under the selected-blocks-and-causal
+    token mask; backward == autograd of the same."""
+    p = make_problem(seed_base=zlib.crc32(name.encode()) % 983, causal=True, **CAUSAL_CASES[name])
+    _compare_fwd(p)
+    o = oracle.Oracle(p)
+    out, lse, _ = o.fwd()
+    dq, dk, dv, fl = o.bwd(out, p.dout, lse)
+    rq, rk, rv = tr.grads(p, p.dout)
+    assert fl == 0
+    for a, r in ((dq, rq), (dk, rk), (dv, rv)):
+        assert torch.allclose(a, r, atol=1e-10, rtol=0), (a - r).abs().max()
+
+
+def test_causal_row_that_sees_nothing_is_empty():
+    """A query block whose only selected kv block lies wholly after its rows
+    sees no token under the mask: out 0, lse -inf (and zero gradients)."""
+    def hook(rng, b, hi, i, sel):
+        return [3] if i == 0 else sel
+    p = make_problem(B=1, N1=1, N2=1, D=16, Sq=256, BQ=64, BKV=64, pattern=pat_causal,
+                     row_hook=hook, seed_base=29, causal=True)
+    o = oracle.Oracle(p)
+    out, lse, fl = o.fwd()
+    assert fl == 0
+    assert torch.all(lse[0, 0, :64] == float("-inf")) and torch.all(out[0, 0, :64] == 0)
+    assert torch.all(torch.isfinite(lse[0, 0, 64:]))
+    dq, dk, dv, _ = o.bwd(out, p.dout, lse)
+    assert torch.all(dq[0, 0, :64] == 0)
+
+
+def test_causal_backward_finite_differences():
+    """Central differences of L = sum(dOut * out) under the causal mask."""
+    p = make_problem(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=8, BQ=4, BKV=4,
+                     lens_q=[9, 12], lens_kv=[14, 12], pattern=pat_random_k, seed_base=31,
+                     dtype=torch.float64, causal=True)
+    dout = p.dout.double()
+
+    def loss(**kw):
+        out, _, _ = oracle.Oracle(p, **kw).fwd()
+        return float((out * dout).sum())
+
+    o = oracle.Oracle(p)
+    out, lse, _ = o.fwd()
+    dq, dk, dv, _ = o.bwd(out, dout, lse)
+    rng = np.random.default_rng(1)
+    eps = 1e-6
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        base = getattr(p, name).double()
+        for _ in range(6):
+            pos = tuple(int(rng.integers(0, s)) for s in base.shape)
+            plus, minus = base.clone(), base.clone()
+            plus[pos] += eps
+            minus[pos] -= eps
+            args = {"q": p.q.double(), "k": p.k.double(), "v": p.v.double()}
+            args[name] = plus
+            lp = loss(**args)
+            args[name] = minus
+            lm = loss(**args)
+            fd = (lp - lm) / (2 * eps)
+            assert abs(fd - float(grad[pos])) <= 1e-6 * max(1.0, abs(fd)), (name, pos, fd, float(grad[pos]))

@@ -63,6 +63,11 @@ def token_mask(p, b):
             for e in row:
                 if e != 0xFFFF:
                     m[h1, i * p.BQ:(i + 1) * p.BQ, int(e) * p.BKV:(int(e) + 1) * p.BKV] = True
+    if getattr(p, "causal", False):
+        # the causal mask, aligned to the end of the kv sequence
+        t = torch.arange(L).view(L, 1)
+        u = torch.arange(kvlen).view(1, kvlen)
+        m &= (u <= t + (kvlen - L)).unsqueeze(0)
     return m
 
 

@@ -49,6 +49,7 @@ class Problem:
     page_size: int = 0
     lens_q: List[int] = field(default_factory=list)
     lens_kv: List[int] = field(default_factory=list)
+    causal: bool = False     # kv token u visible to query row t iff u <= t + kvlen - qlen
 
     @property
     def W(self) -> int:
@@ -59,7 +60,8 @@ class Problem:
                 "B": self.B, "N1": self.N1, "N2": self.N2, "D": self.D,
                 "dtype": str(self.dtype).replace("torch.", ""),
                 "block_shape": [self.BQ, self.BKV], "Hidx": self.Hidx, "W": self.W,
-                "lens_q": self.lens_q, "lens_kv": self.lens_kv, "page_size": self.page_size}
+                "lens_q": self.lens_q, "lens_kv": self.lens_kv, "page_size": self.page_size,
+                "causal": self.causal}
 
 
 # ----------------------------------------------------------------------------
@@ -90,6 +92,12 @@ def pat_fraction_diag(frac):
 
 def pat_dense(rng, i, nq, nk):
     return list(range(nk))
+
+
+def pat_causal(rng, i, nq, nk):
+    """Every block a causal row can reach (query and kv blocks of equal size,
+    the kv sequence ending where the query sequence ends)."""
+    return list(range(min(nk, i + 1 + max(0, nk - nq))))
 
 
 def pat_sink_diag_random(extra):
@@ -136,7 +144,7 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
                  Sq=None, Skv=None, kv_storage=None, Hidx=None, W=None,
                  pattern: Callable = pat_random_k, page_size=128, extra_pages=0,
                  use_seqused_kv=None, seed_base=0, scale=None, max_pages=None,
-                 row_hook: Optional[Callable] = None) -> Problem:
+                 row_hook: Optional[Callable] = None, causal: bool = False) -> Problem:
     """Build one seeded problem.
 
     lens_q / lens_kv: per-batch valid lengths (TND q: the stored lengths).
@@ -224,7 +232,7 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
                    dtype=dtype, BQ=BQ, BKV=BKV, Hidx=Hidx, scale=scale, q=q, k=k, v=v,
                    dout=dout, index=index, cu_q=cu_q, cu_kv=cu_kv, seqused_kv=seqused,
                    block_table=block_table, page_size=(page_size if layout_kv == "PA_BBND" else 0),
-                   lens_q=lens_q, lens_kv=lens_kv)
+                   lens_q=lens_q, lens_kv=lens_kv, causal=causal)
 
 
 # ----------------------------------------------------------------------------
