@@ -10,7 +10,7 @@ the backward consuming the forward's out and lse.  Effective FLOPs count
 kept (q head, valid q token, valid kv token) pairs only: 4*D per pair
 forward, 10*D backward.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C3] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config C3] [--causal] [--impl ours|reference]
 
 Under torchrun each rank runs an independent replica of the workload on its
 own GPU (the path shards by batch / kv-head group with no exchange), so the
@@ -56,36 +56,39 @@ def _peaks():
 
 
 def _pairs(p):
-    from workloads.gen import NO_BLOCK  # noqa: F401  (structure only)
     # kept pairs = sum over (head, query block row) of valid q rows x valid
-    # kv tokens of the accepted blocks; the index of every workload here is
-    # valid (ascending, in range), so accepted = present entries
+    # kv tokens of the accepted blocks (causal: only the tokens each row
+    # sees); the index of every workload here is valid (ascending, in
+    # range), so accepted = present entries
     idx = p.index.view(torch.int16).numpy().view(np.uint16).astype(np.int64)
     g = p.N1 // p.N2
+    heads = 1 if p.Hidx == p.N1 else g
+    causal = bool(getattr(p, "causal", False))
+
+    def row_pairs(b, i, e):
+        e = e[e != 0xFFFF]
+        rows = min(p.BQ, p.lens_q[b] - i * p.BQ)
+        lo = e * p.BKV
+        hi = np.minimum(lo + p.BKV, p.lens_kv[b])
+        if not causal:
+            return rows * int((hi - lo).sum())
+        t = i * p.BQ + np.arange(rows, dtype=np.int64)
+        last = t[None, :] + (p.lens_kv[b] - p.lens_q[b]) + 1   # one past the last token row t sees
+        return int(np.maximum(0, np.minimum(hi[:, None], last) - lo[:, None]).sum())
+
     total = 0
-    lens_q, lens_kv = p.lens_q, p.lens_kv
     if p.layout_q == "BNSD":
         for b in range(p.B):
             for hi in range(p.Hidx):
-                heads = 1 if p.Hidx == p.N1 else g
                 for i in range(idx.shape[2]):
-                    rows = min(p.BQ, lens_q[b] - i * p.BQ)
-                    e = idx[b, hi, i]
-                    e = e[e != 0xFFFF]
-                    cols = int(np.minimum(p.BKV, lens_kv[b] - e * p.BKV).sum())
-                    total += heads * rows * cols
+                    total += heads * row_pairs(b, i, idx[b, hi, i])
     else:
         off = 0
         for b in range(p.B):
-            nq = -(-lens_q[b] // p.BQ)
+            nq = -(-p.lens_q[b] // p.BQ)
             for hi in range(p.Hidx):
-                heads = 1 if p.Hidx == p.N1 else g
                 for i in range(nq):
-                    rows = min(p.BQ, lens_q[b] - i * p.BQ)
-                    e = idx[hi, off + i]
-                    e = e[e != 0xFFFF]
-                    cols = int(np.minimum(p.BKV, lens_kv[b] - e * p.BKV).sum())
-                    total += heads * rows * cols
+                    total += heads * row_pairs(b, i, idx[hi, off + i])
             off += nq
     return total
 
@@ -143,23 +146,28 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- oracle leg
-def _oracle_subproblem(cfg: int, q_rows: int):
+def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False):
     """A bounded slice of the workload for the CPU oracle: batch 0, head 0,
-    the first q_rows query rows against the full key range."""
+    the first q_rows query rows against the full key range (causal: the
+    last q_rows rows, which keeps every row's place relative to the end of
+    the kv sequence)."""
     import workloads
     from workloads.gen import make_problem, pat_dense
-    p = workloads.make_config(cfg)
+    p = workloads.make_config(cfg, causal=causal)
     if p.layout_q != "BNSD":
         raise SystemExit("CPU baseline slice is defined for the BNSD workloads")
     S = p.q.shape[2]
     q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
     sub = make_problem(B=1, N1=1, N2=1, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
-                       BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale)
-    sub.q = p.q[:1, :1, :q_rows].contiguous()
+                       BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale,
+                       causal=causal)
+    rows = slice(S - q_rows, S) if causal else slice(0, q_rows)
+    blocks = slice(rows.start // p.BQ, rows.stop // p.BQ)
+    sub.q = p.q[:1, :1, rows].contiguous()
     sub.k = p.k[:1, :1].contiguous()
     sub.v = p.v[:1, :1].contiguous()
-    sub.dout = p.dout[:1, :1, :q_rows].contiguous()
-    sub.index = p.index[:1, :1, :q_rows // p.BQ].contiguous()
+    sub.dout = p.dout[:1, :1, rows].contiguous()
+    sub.index = p.index[:1, :1, blocks].contiguous()
     sub.lens_q = [q_rows]
     return sub
 
@@ -173,21 +181,26 @@ def _oracle_step(sub):
     return time.perf_counter() - t
 
 
-def _oracle_rate(cfg: int, target_s: float):
-    """Calibrate the slice to ~target_s per step; returns (sub, pairs, seconds)."""
-    sub = _oracle_subproblem(cfg, 128)
+def _oracle_rate(cfg: int, target_s: float, causal: bool = False):
+    """Calibrate the slice to ~target_s per step; returns (sub, pairs)."""
+    sub = _oracle_subproblem(cfg, 128, causal)
     t = _oracle_step(sub)
     rows = int(128 * max(1.0, target_s / max(t, 1e-3)))
-    sub = _oracle_subproblem(cfg, rows)
+    sub = _oracle_subproblem(cfg, rows, causal)
     return sub, _pairs(sub)
 
 
-def cpu_baseline(cfg: int, target_s: float = 12.0):
-    sub, pairs = _oracle_rate(cfg, target_s)
+def _descr(cfg: int, causal: bool) -> str:
+    return DESCR[cfg] + (", causal mask + lower-triangular index" if causal else "")
+
+
+def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False):
+    sub, pairs = _oracle_rate(cfg, target_s, causal)
     t = _oracle_step(sub)
     flops = 14 * sub.D * pairs
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _omp_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle fwd+bwd on batch 0, head 0, first {sub.q.shape[2]} query rows "
+            "sample": f"fp64 oracle fwd+bwd on batch 0, head 0, {'last' if causal else 'first'} "
+                      f"{sub.q.shape[2]} query rows "
                       f"x {sub.k.shape[2]} keys of {DESCR[cfg].split(':')[0]} ({pairs} kept pairs, "
                       f"{t:.1f} s)"}
 
@@ -201,7 +214,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    sub, pairs = _oracle_rate(args.config, 2.0)
+    sub, pairs = _oracle_rate(args.config, 2.0, args.causal)
     for _ in range(args.warmup):
         _oracle_step(sub)
     ts = [_oracle_step(sub) for _ in range(args.steps)]
@@ -212,10 +225,11 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": DESCR[args.config], "sample": "see cpu_baseline"},
+            "config": {"workload": _descr(args.config, args.causal), "sample": "see cpu_baseline"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _omp_threads(),
                              "kind": "oracle",
-                             "sample": f"batch 0, head 0, first {sub.q.shape[2]} query rows "
+                             "sample": f"batch 0, head 0, {'last' if args.causal else 'first'} "
+                                       f"{sub.q.shape[2]} query rows "
                                        f"({pairs} kept pairs) per step"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -258,7 +272,7 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    p = workloads.make_config(args.config, args.batch)
+    p = workloads.make_config(args.config, args.batch, args.causal)
     pairs = _pairs(p)
     P = params_of(p)
     to = lambda t: None if t is None else t.to(dev)  # noqa: E731
@@ -361,14 +375,14 @@ def run_ours(args):
         peak = peaks["bf16_tflops"]
         dominant = "bwd" if bwd_kms >= fwd_kms else "fwd"
         achieved = bwd_ktf if dominant == "bwd" else fwd_ktf
-        traffic = _traffic_from_profiles(args.config, dominant)
+        traffic = None if args.causal else _traffic_from_profiles(args.config, dominant)
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if p.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-            "config": {"workload": DESCR[args.config] if args.batch is None
-                       else DESCR[args.config] + f" (batch overridden to {args.batch})",
+            "config": {"workload": _descr(args.config, args.causal) if args.batch is None
+                       else _descr(args.config, args.causal) + f" (batch overridden to {args.batch})",
                        "kept_pairs_per_replica": pairs,
                        "parallelism": f"replicas x{world} (no exchange)",
                        "l2": "inputs larger than L2 (q/k/v/dout %d MiB each)"
@@ -392,7 +406,7 @@ def run_ours(args):
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(args.config)
+            line["cpu_baseline"] = cpu_baseline(args.config, causal=args.causal)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -420,7 +434,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="smaller batch for C3/C4 (profiler captures only; not a bench line)")
+    ap.add_argument("--causal", action="store_true",
+                    help="C3 with the causal mask and its lower-triangular block index")
     args = ap.parse_args()
+    if args.causal and args.config != 3:
+        ap.error("--causal applies to C3")
     if args.impl == "reference":
         run_reference(args)
     else:

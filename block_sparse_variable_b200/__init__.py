@@ -46,7 +46,7 @@ class bsa_params(ctypes.Structure):
     _fields_ = [("q_layout", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
                 ("num_heads", ctypes.c_int64), ("num_kv_heads", ctypes.c_int64),
                 ("block_shape", ctypes.c_int64 * 2), ("scale", ctypes.c_double),
-                ("return_lse", ctypes.c_int32)]
+                ("return_lse", ctypes.c_int32), ("mask_type", ctypes.c_int32)]
 
 
 class bsa_ws_region(ctypes.Structure):
@@ -111,6 +111,7 @@ class Params:
     block_shape: Tuple[int, int] = (128, 128)
     scale: float = 0.0
     return_lse: bool = True
+    causal: bool = False
 
     def c(self) -> bsa_params:
         p = bsa_params()
@@ -119,6 +120,7 @@ class Params:
         p.block_shape[0], p.block_shape[1] = self.block_shape
         p.scale = float(self.scale)
         p.return_lse = 1 if self.return_lse else 0
+        p.mask_type = 1 if self.causal else 0
         return p
 
 
@@ -172,9 +174,10 @@ def _stream(stream) -> Optional[int]:
 
 
 def params_for(q_layout, kv_layout, num_heads, num_kv_heads=0, block_shape=(128, 128), scale=0.0,
-               return_lse=True) -> Params:
+               return_lse=True, causal=False) -> Params:
     return Params(q_layout, kv_layout, int(num_heads), int(num_kv_heads),
-                  (int(block_shape[0]), int(block_shape[1])), float(scale), bool(return_lse))
+                  (int(block_shape[0]), int(block_shape[1])), float(scale), bool(return_lse),
+                  bool(causal))
 
 
 def _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table, out, lse):

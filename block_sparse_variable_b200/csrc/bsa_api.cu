@@ -183,6 +183,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   if (W < 1 || W > 65535 || R < 0 || ix->stride[ix->ndim - 1] != 1) return BSA_ERR_PARAM_INVALID;
 
   // lse
+  if (P.mask_type != BSA_MASK_NONE && P.mask_type != BSA_MASK_CAUSAL) return BSA_ERR_PARAM_INVALID;
   const bool want_lse = a.bwd || P.return_lse;
   if (want_lse) {
     if (!present(a.lse)) return BSA_ERR_NULLPTR;
@@ -231,6 +232,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   p.scale = float(scale);
   p.scale_log2 = float(scale * 1.4426950408889634);
   p.return_lse = want_lse ? 1 : 0;
+  p.causal = P.mask_type == BSA_MASK_CAUSAL ? 1 : 0;
   p.fwd_slots = fwd_slots; p.bwd_slots = bwd_slots;
   p.fwd_slots_pad = fpad; p.bwd_slots_pad = bpad;
 
@@ -396,7 +398,7 @@ bsa_status bsa_set_main_kernel_events(void *before, void *after) {
   return BSA_OK;
 }
 
-int32_t bsa_abi_version(void) { return 1; }
+int32_t bsa_abi_version(void) { return 2; }
 
 const char *bsa_status_string(bsa_status s) {
   switch (s) {

@@ -47,6 +47,7 @@ struct Problem {
   int64_t rows_q;   // q storage rows: B*Sq (BNSD) or Tq (TND)
   float scale, scale_log2;  // scale, scale * log2(e)
   int32_t return_lse;
+  int32_t causal;  // kv token u visible to query row t iff u <= t + kvlen - qlen
 
   // ---- tensors (strides in elements).  Token row t of batch b, head h:
   //   base + b*sb + (tok0_b + t)*st + h*sh   (tok0 = 0 for BNSD, cu[b] for TND)

@@ -33,7 +33,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
+#include <type_traits>
 
 #include "addr.cuh"
 #include "bsa_internal.h"
@@ -423,7 +425,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const float *lse2 = stat + slot * 256;
         const float *dsum = lse2 + 128;
         uint32_t pp[32], dd[32];
-        {
+        // causal: column q (query row t0 + q) sees this kv row iff q >= qmin;
+        // the masked variant runs only where a warp's columns cross the diagonal
+        const int qmin = p.causal ? v.u0 + r - (v.kvlen - v.bi.qlen) - t0 : INT_MIN;
+        auto softmax = [&](auto masked) {
           // 16-column blocks of S^T and dP^T, the next block's TMEM loads in
           // flight while this one is computed
           const uint32_t c0 = uint32_t(64 * wg);
@@ -441,8 +446,12 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
             for (int c2 = 0; c2 < 16; c2 += 2) {
               const int q = int(c0) + 16 * k + c2;
-              const float p0 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2]), p.scale_log2, -lse2[q])) : 0.f;
-              const float p1 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
+              float p0 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2]), p.scale_log2, -lse2[q])) : 0.f;
+              float p1 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
+              if constexpr (decltype(masked)::value) {
+                p0 = q >= qmin ? p0 : 0.f;
+                p1 = q + 1 >= qmin ? p1 : 0.f;
+              }
               const float s0 = p0 * (__uint_as_float(bd[c2]) - dsum[q]);
               const float s1 = p1 * (__uint_as_float(bd[c2 + 1]) - dsum[q + 1]);
               pp[8 * k + (c2 >> 1)] = MmaOp<T>::pack(p0, p1);
@@ -450,7 +459,11 @@ __global__ void __launch_bounds__(kBThreads, 1)
             }
             if (k + 1 < 4) tmem_wait_ld();
           }
-        }
+        };
+        if (__any_sync(0xffffffffu, qmin > 64 * wg))
+          softmax(std::true_type{});
+        else
+          softmax(std::false_type{});
         // P and dS into this group's own R0 columns (no other group reads
         // them as S), dS also into shared memory for the dQ product
         tmem_st32(tR0 + lane_off + uint32_t(64 * wg), pp);

@@ -385,6 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the chunk walk needs only the index row, its length, kvlen and the
         // batch; the rest of the item is re-derived for the epilogue
         ItemView v;
+        int coff;  // causal: the last kv token this row sees, else beyond all
         {
           const ItemView full = item_view(p, p.fwd_items[it]);
           v.crow = full.crow;
@@ -393,6 +394,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v.b = full.b;
           v.ksl = p.ksl;
           v.BKV = p.BKV;
+          coff = p.causal ? full.t0 + r + full.kvlen - full.bi.qlen : (1 << 30);
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
              ch = next_chunk(p, v, ch), ++n, ++kv_it) {
@@ -400,8 +402,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (!(ok = wait_warp(bar(kBarSFull + b), (kv_it / kSBufs) & 1u, abort, p.status))) break;
           tc_fence_after();
           const uint32_t tS = tS0 + uint32_t(b) * 128u + lane_off;
-          const int valid_all = v.kvlen - v.u0(ch);       // kv columns of the chunk that exist
-          const int valid = valid_all - kCols * wg;        // of this group's columns
+          const int u0c = v.u0(ch);
+          const int valid_all = v.kvlen - u0c;             // kv columns of the chunk that exist
+          // the chunk columns this row may see (causal: up to its own token)
+          const int vis_all = min(valid_all, coff - u0c + 1);
+          const int valid = vis_all - kCols * wg;          // of this group's columns
           if (valid_all < 128) {
             // kv rows past the used length may hold anything (the rest of a
             // page, another sequence's tokens, even NaN); their P is (nearly)
@@ -459,9 +464,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // out to change little, which is still exact); no max is needed.
           // (the first chunk of an item always takes a reference: both groups
           // know that without exchanging flags)
+          // (a row whose visible scores are all still masked keeps m = -inf
+          // and always asks for a reference)
           uint32_t any = 1;
-          if (!first) {
-            const uint32_t need = __any_sync(0xffffffffu, !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
+          if (n > 0) {
+            const uint32_t need =
+                __any_sync(0xffffffffu, first || !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
             if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
             if (!rendezvous()) break;
             // one decision for the rows of this warp, shared with the other
@@ -484,7 +492,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 uint32_t y[kCols / 2];
                 tmem_ld_cols<kCols / 2>(tS + uint32_t(kCols * g2 + (kCols / 2) * h), y);
                 tmem_wait_ld();
-                const int vy = valid_all - kCols * g2 - (kCols / 2) * h;
+                const int vy = vis_all - kCols * g2 - (kCols / 2) * h;
 #pragma unroll
                 for (int c = 0; c < kCols / 2; ++c)
                   if (c < vy) ym = fmaxf(ym, __uint_as_float(y[c]));
@@ -496,14 +504,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float m_new = fmaxf(m, cm);
             alpha = first ? 1.f : ex2(m - m_new);
             m = m_new;
-            exps(m);
+            exps(m > -INFINITY ? m : 0.f);  // nothing visible yet: every P is 0
           }
           // P over the first half of this group's own S columns: no other
           // warp reads them any more (the grow path's reads of the other
           // group's S precede its rendezvous)
           tmem_st_cols<kCols / 2>(tS + uint32_t(kCols * wg), pk);
           l = l * alpha + (ps[0] + ps[1]);
-          if (grow && !first && __any_sync(0xffffffffu, alpha != 1.f)) {
+          if (grow && __any_sync(0xffffffffu, !first && alpha != 1.f)) {
             // O may only be rescaled once P_{t-1} V_{t-1} (and so every
             // earlier product, the tensor pipe being in order) has landed
             const uint32_t t = kv_it - 1;

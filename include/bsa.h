@@ -85,7 +85,16 @@ typedef struct bsa_params {
   int64_t block_shape[2]; /* {BQ, BKV}, each in {128, 256, 512, 1024} */
   double scale;           /* 0 means 1/sqrt(D) */
   int32_t return_lse;     /* forward only: write lse when non-zero */
+  int32_t mask_type;      /* BSA_MASK_NONE or BSA_MASK_CAUSAL */
 } bsa_params;
+
+/* Token mask inside the selected blocks (GenericBlockSparseAttention article,
+ * mask section: a built-in causal mode).  BSA_MASK_CAUSAL keeps kv token u for
+ * query row t of batch b only when u <= t + kvlen_b - qlen_b: the mask is
+ * aligned to the end of the kv sequence (the page does not state the
+ * alignment; this is our reading, the usual one when a query chunk continues
+ * a longer kv sequence).  A row that keeps no token gives out 0, lse -inf. */
+enum { BSA_MASK_NONE = 0, BSA_MASK_CAUSAL = 1 };
 
 /* Status codes: the first three echo the aclnn codes the pages list
  * (161001 null pointer, 161002 invalid parameter, 561103 inner error). */
@@ -281,7 +290,8 @@ bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64
  * Asynchronous on `stream`; BSA_ERR_NULLPTR for a NULL flags pointer. */
 bsa_status bsa_selftest_wait_timeout(uint32_t *flags, void *stream);
 
-/* Library ABI version (bumped on any signature or layout change). */
+/* Library ABI version (bumped on any signature or layout change; 2 added
+ * bsa_params.mask_type). */
 int32_t bsa_abi_version(void);
 
 #ifdef __cplusplus

@@ -25,7 +25,7 @@ def test_exports_every_declared_symbol():
     for n in names:
         assert hasattr(bsa.lib(), n), n
     assert set(names) == set(bsa.EXPORTED)
-    assert bsa.lib().bsa_abi_version() == 1
+    assert bsa.lib().bsa_abi_version() == 2
 
 
 def test_status_strings():
@@ -152,3 +152,20 @@ def test_empty_query_is_a_no_op():
                               lse=torch.empty(0, p.N1), workspace=torch.zeros(256, dtype=torch.uint8),
                               stream=0)
     assert out.numel() == 0
+
+
+def test_mask_type_must_be_known():
+    """bsa_params.mask_type is BSA_MASK_NONE (0) or BSA_MASK_CAUSAL (1)."""
+    import dataclasses
+    p = _prob()
+    P = params_of(p)
+
+    class Bad(bsa.Params):
+        def c(self):
+            c = super().c()
+            c.mask_type = 7
+            return c
+
+    bad = Bad(**{f.name: getattr(P, f.name) for f in dataclasses.fields(P)})
+    assert _code(lambda: _ws(p, params=bad)) == 161002
+    assert _ws(p, params=dataclasses.replace(P, causal=True)) == _ws(p)

@@ -74,8 +74,32 @@ EDGE = {
 }
 
 
+# causal mask aligned to the end of the kv sequence: query row t sees kv
+# token u iff u <= t + kvlen - qlen (rows with nothing visible: lse -inf, out 0)
+CAUSAL = {
+    "causal_bnsd_dense": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=128, Sq=640,
+                              pattern=pat_dense, causal=True),
+    "causal_bnsd_128x512": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=1, D=64, Sq=1100,
+                                BKV=512, pattern=pat_dense, causal=True),
+    "causal_bnsd_ragged_kv": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=2, D=64, Sq=300,
+                                  lens_kv=[300, 470], Skv=470, pattern=pat_dense, causal=True),
+    "causal_tnd_gqa_prefix": dict(layout_q="TND", layout_kv="TND", B=3, N1=4, N2=2, D=64,
+                                  lens_q=[130, 300, 77], lens_kv=[400, 300, 205],
+                                  pattern=pat_random_k, causal=True),
+    "causal_tnd_q_longer": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=128,
+                                lens_q=[300, 140], lens_kv=[150, 140], pattern=pat_dense,
+                                causal=True),
+    "causal_tnd_fp16_256x256": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=2, D=128,
+                                    BQ=256, BKV=256, lens_q=[700, 260], lens_kv=[700, 500],
+                                    dtype=torch.float16, pattern=pat_density(0.7, 1), causal=True),
+    "causal_paged": dict(layout_q="TND", layout_kv="PA_BBND", B=3, N1=4, N2=2, D=64,
+                         lens_q=[200, 129, 64], lens_kv=[456, 129, 300], page_size=128,
+                         extra_pages=2, pattern=pat_dense, causal=True),
+}
+
+
 def _problem(name):
-    spec = dict(SMALL.get(name) or EDGE[name])
+    spec = dict(SMALL.get(name) or EDGE.get(name) or CAUSAL[name])
     return make_problem(seed_base=zlib.crc32(name.encode()) % 9973, name=name, **spec)
 
 
@@ -152,6 +176,13 @@ def test_small_cases(name):
 @pytest.mark.parametrize("name", sorted(EDGE))
 def test_edge_cases(name):
     _run_and_check(_problem(name))
+
+
+@pytest.mark.parametrize("name", sorted(CAUSAL))
+def test_causal_cases(name):
+    p = _problem(name)
+    assert p.causal
+    _run_and_check(p)
 
 
 def _poison_unused_kv(p):

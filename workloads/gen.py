@@ -100,6 +100,14 @@ def pat_causal(rng, i, nq, nk):
     return list(range(min(nk, i + 1 + max(0, nk - nq))))
 
 
+def pat_causal_blocks(BQ, BKV):
+    """Every kv block of BKV tokens that a causal row of query block i (BQ
+    rows) can reach, with query and kv sequences of one length."""
+    def f(rng, i, nq, nk):
+        return list(range(min(nk, (i * BQ + BQ - 1) // BKV + 1)))
+    return f
+
+
 def pat_sink_diag_random(extra):
     """block 0, the diagonal block i and `extra` distinct random blocks from [1, i-1]."""
     def f(rng, i, nq, nk):
@@ -243,13 +251,16 @@ def _lens(seed, B, lo, hi):
     return [int(x) for x in rng.integers(lo, hi + 1, size=B)]
 
 
-def make_config(c: int, batch: int | None = None) -> Problem:
+def make_config(c: int, batch: int | None = None, causal: bool = False) -> Problem:
     """C1..C5: the five workload shapes (see the module docstring for seeds).
 
     `batch` overrides the batch of the BNSD shapes C3 and C4 (smaller cases
-    of the same kernels for profiler captures)."""
+    of the same kernels for profiler captures).  `causal` turns C3 into its
+    causal variant: the causal mask with the lower-triangular block index."""
     if batch is not None and c not in (3, 4):
         raise ValueError("batch override applies to C3 and C4 only")
+    if causal and c != 3:
+        raise ValueError("the causal variant is defined for C3 only")
     s = 1000 * c
     if c == 1:
         return make_problem(name="C1", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=64,
@@ -261,8 +272,10 @@ def make_config(c: int, batch: int | None = None) -> Problem:
                             pattern=pat_fraction_diag(0.25), W=max(math.ceil(l / 128) for l in lens),
                             seed_base=s)
     if c == 3:
-        return make_problem(name="C3", layout_q="BNSD", layout_kv="BNSD", B=batch or 2, N1=32, N2=32, D=128,
-                            Sq=8192, BQ=128, BKV=512, W=16, pattern=pat_dense, seed_base=s)
+        return make_problem(name="C3-causal" if causal else "C3", layout_q="BNSD", layout_kv="BNSD",
+                            B=batch or 2, N1=32, N2=32, D=128, Sq=8192, BQ=128, BKV=512, W=16,
+                            pattern=pat_causal_blocks(128, 512) if causal else pat_dense,
+                            seed_base=s, causal=causal)
     if c == 4:
         return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=batch or 1, N1=24, N2=24, D=128,
                             Sq=32768, BQ=128, BKV=128, W=256, pattern=pat_sink_diag_random(14),
