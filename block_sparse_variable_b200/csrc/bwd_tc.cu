@@ -154,7 +154,7 @@ __device__ __forceinline__ int b_t0(const Problem &p, const BItem &v, const BSte
   return b_qblock(p, v, c.hh, c.e, TK) * p.BQ + c.st * 128;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kCausal>
 __global__ void __launch_bounds__(kBThreads, 1)
     k_bwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         uint32_t pp[32], dd[32];
         // causal: column q (query row t0 + q) sees this kv row iff q >= qmin;
         // the masked variant runs only where a warp's columns cross the diagonal
-        const int qmin = p.causal ? v.u0 + r - (v.kvlen - v.bi.qlen) - t0 : INT_MIN;
+        const int qmin = kCausal ? v.u0 + r - (v.kvlen - v.bi.qlen) - t0 : INT_MIN;
         auto softmax = [&](auto masked) {
           // 16-column blocks of S^T and dP^T, the next block's TMEM loads in
           // flight while this one is computed
@@ -460,10 +460,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
             if (k + 1 < 4) tmem_wait_ld();
           }
         };
-        if (__any_sync(0xffffffffu, qmin > 64 * wg))
-          softmax(std::true_type{});
-        else
+        if constexpr (kCausal) {
+          if (__any_sync(0xffffffffu, qmin > 64 * wg))
+            softmax(std::true_type{});
+          else
+            softmax(std::false_type{});
+        } else {
           softmax(std::false_type{});
+        }
         // P and dS into this group's own R0 columns (no other group reads
         // them as S), dS also into shared memory for the dQ product
         tmem_st32(tR0 + lane_off + uint32_t(64 * wg), pp);
@@ -564,14 +568,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kCausal>
 cudaError_t launch_bwd_tc(const Problem &p, const BwdMaps &m, cudaStream_t s) {
   const int smem = BLayout<D>::kBytes > 120 * 1024 ? BLayout<D>::kBytes : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<D, BF16, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.bwd_slots < num_sms() ? p.bwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_bwd_tc<D, BF16><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
+  k_bwd_tc<D, BF16, kCausal><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
   return cudaGetLastError();
 }
 
@@ -581,9 +585,16 @@ cudaError_t launch_bwd_main(const Problem &p, cudaStream_t s) {
   BwdMaps m;
   cudaError_t e = make_bwd_maps(p, m);
   if (e != cudaSuccess) return e;
+  // the causal mask is a separate instantiation: the unmasked kernel carries
+  // none of its arithmetic
+  if (p.causal) {
+    if (p.dtype == BSA_BF16)
+      return p.D == 64 ? launch_bwd_tc<64, true, true>(p, m, s) : launch_bwd_tc<128, true, true>(p, m, s);
+    return p.D == 64 ? launch_bwd_tc<64, false, true>(p, m, s) : launch_bwd_tc<128, false, true>(p, m, s);
+  }
   if (p.dtype == BSA_BF16)
-    return p.D == 64 ? launch_bwd_tc<64, true>(p, m, s) : launch_bwd_tc<128, true>(p, m, s);
-  return p.D == 64 ? launch_bwd_tc<64, false>(p, m, s) : launch_bwd_tc<128, false>(p, m, s);
+    return p.D == 64 ? launch_bwd_tc<64, true, false>(p, m, s) : launch_bwd_tc<128, true, false>(p, m, s);
+  return p.D == 64 ? launch_bwd_tc<64, false, false>(p, m, s) : launch_bwd_tc<128, false, false>(p, m, s);
 }
 
 }  // namespace bsa

@@ -176,7 +176,7 @@ __device__ __forceinline__ ItemView item_view(const Problem &p, int id) {
   return v;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kCausal>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_fwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         // the chunk walk needs only the index row, its length, kvlen and the
         // batch; the rest of the item is re-derived for the epilogue
         ItemView v;
-        int coff;  // causal: the last kv token this row sees, else beyond all
+        int coff;  // causal: the last kv token this row sees
         {
           const ItemView full = item_view(p, p.fwd_items[it]);
           v.crow = full.crow;
@@ -394,7 +394,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           v.b = full.b;
           v.ksl = p.ksl;
           v.BKV = p.BKV;
-          coff = p.causal ? full.t0 + r + full.kvlen - full.bi.qlen : (1 << 30);
+          coff = kCausal ? full.t0 + r + full.kvlen - full.bi.qlen : 0;
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
              ch = next_chunk(p, v, ch), ++n, ++kv_it) {
@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int u0c = v.u0(ch);
           const int valid_all = v.kvlen - u0c;             // kv columns of the chunk that exist
           // the chunk columns this row may see (causal: up to its own token)
-          const int vis_all = min(valid_all, coff - u0c + 1);
+          const int vis_all = kCausal ? min(valid_all, coff - u0c + 1) : valid_all;
           const int valid = vis_all - kCols * wg;          // of this group's columns
           if (valid_all < 128) {
             // kv rows past the used length may hold anything (the rest of a
@@ -467,9 +467,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // (a row whose visible scores are all still masked keeps m = -inf
           // and always asks for a reference)
           uint32_t any = 1;
-          if (n > 0) {
+          if (kCausal ? n > 0 : !first) {
             const uint32_t need =
-                __any_sync(0xffffffffu, first || !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
+                __any_sync(0xffffffffu, (kCausal && first) || !(ps[0] + ps[1] <= kRescaleSum)) ? 1u : 0u;
             if (lane == 0) flags[(kv_it & 1u) * kWarps + warp] = need;
             if (!rendezvous()) break;
             // one decision for the rows of this warp, shared with the other
@@ -504,14 +504,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const float m_new = fmaxf(m, cm);
             alpha = first ? 1.f : ex2(m - m_new);
             m = m_new;
-            exps(m > -INFINITY ? m : 0.f);  // nothing visible yet: every P is 0
+            exps(!kCausal || m > -INFINITY ? m : 0.f);  // nothing visible yet: every P is 0
           }
           // P over the first half of this group's own S columns: no other
           // warp reads them any more (the grow path's reads of the other
           // group's S precede its rendezvous)
           tmem_st_cols<kCols / 2>(tS + uint32_t(kCols * wg), pk);
           l = l * alpha + (ps[0] + ps[1]);
-          if (grow && __any_sync(0xffffffffu, !first && alpha != 1.f)) {
+          if (grow && (kCausal || !first) && __any_sync(0xffffffffu, (!kCausal || !first) && alpha != 1.f)) {
             // O may only be rescaled once P_{t-1} V_{t-1} (and so every
             // earlier product, the tensor pipe being in order) has landed
             const uint32_t t = kv_it - 1;
@@ -587,16 +587,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool kCausal>
 cudaError_t launch_tc(const Problem &p, const FwdMaps &m, cudaStream_t s) {
   // at least 120 KB so that exactly one CTA (the sole owner of all 512 TMEM
   // columns) is resident per SM
   const int smem = Layout<D>::kAlloc > 120 * 1024 ? Layout<D>::kAlloc : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.fwd_slots < num_sms() ? p.fwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_fwd_tc<D, BF16><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
+  k_fwd_tc<D, BF16, kCausal><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
   return cudaGetLastError();
 }
 
@@ -606,9 +606,16 @@ cudaError_t launch_fwd_main(const Problem &p, cudaStream_t s) {
   FwdMaps m;
   cudaError_t e = make_fwd_maps(p, m);
   if (e != cudaSuccess) return e;
+  // the causal mask is a separate instantiation: the unmasked kernel carries
+  // none of its arithmetic
+  if (p.causal) {
+    if (p.dtype == BSA_BF16)
+      return p.D == 64 ? launch_tc<64, true, true>(p, m, s) : launch_tc<128, true, true>(p, m, s);
+    return p.D == 64 ? launch_tc<64, false, true>(p, m, s) : launch_tc<128, false, true>(p, m, s);
+  }
   if (p.dtype == BSA_BF16)
-    return p.D == 64 ? launch_tc<64, true>(p, m, s) : launch_tc<128, true>(p, m, s);
-  return p.D == 64 ? launch_tc<64, false>(p, m, s) : launch_tc<128, false>(p, m, s);
+    return p.D == 64 ? launch_tc<64, true, false>(p, m, s) : launch_tc<128, true, false>(p, m, s);
+  return p.D == 64 ? launch_tc<64, false, false>(p, m, s) : launch_tc<128, false, false>(p, m, s);
 }
 
 }  // namespace bsa
