@@ -42,8 +42,11 @@ DESCR = {
     4: "C4: BNSD B=1 N1=N2=24 S=32768 D=128 bf16, block (128,128), sink+diag+14 random of 256",
     5: "C5: TND q B=8 lens U[512,4096] + paged KV [P,128,8,128] fp16, N1=32 N2=8, top-8 blocks",
 }
-# kernels this library launches per step (forward 5, backward 12)
+# kernels this library launches per step (forward 5, backward 12; the
+# deterministic backward 14: the forward list's sort and the dQ pass added,
+# the dQ conversion dropped)
 LAUNCHES_PER_STEP = 17
+LAUNCHES_PER_STEP_DET = 19
 
 
 def _peaks():
@@ -190,8 +193,9 @@ def _oracle_rate(cfg: int, target_s: float, causal: bool = False):
     return sub, _pairs(sub)
 
 
-def _descr(cfg: int, causal: bool) -> str:
-    return DESCR[cfg] + (", causal mask + lower-triangular index" if causal else "")
+def _descr(cfg: int, causal: bool, deterministic: bool = False) -> str:
+    return (DESCR[cfg] + (", causal mask + lower-triangular index" if causal else "")
+            + (", deterministic backward" if deterministic else ""))
 
 
 def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False):
@@ -273,6 +277,7 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
 
     p = workloads.make_config(args.config, args.batch, args.causal)
+    p.deterministic = args.deterministic
     pairs = _pairs(p)
     P = params_of(p)
     to = lambda t: None if t is None else t.to(dev)  # noqa: E731
@@ -375,24 +380,26 @@ def run_ours(args):
         peak = peaks["bf16_tflops"]
         dominant = "bwd" if bwd_kms >= fwd_kms else "fwd"
         achieved = bwd_ktf if dominant == "bwd" else fwd_ktf
-        traffic = None if args.causal else _traffic_from_profiles(args.config, dominant)
+        traffic = (None if args.causal or args.deterministic
+                   else _traffic_from_profiles(args.config, dominant))
+        bwd_name = "k_bwd_tc+k_dq_tc" if args.deterministic else "k_bwd_tc"
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if p.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-            "config": {"workload": _descr(args.config, args.causal) if args.batch is None
-                       else _descr(args.config, args.causal) + f" (batch overridden to {args.batch})",
+            "config": {"workload": _descr(args.config, args.causal, args.deterministic)
+                       + ("" if args.batch is None else f" (batch overridden to {args.batch})"),
                        "kept_pairs_per_replica": pairs,
                        "parallelism": f"replicas x{world} (no exchange)",
                        "l2": "inputs larger than L2 (q/k/v/dout %d MiB each)"
                              % (q.numel() * q.element_size() >> 20)},
             "fwd_ms": round(fwd_ms, 4), "bwd_ms": round(bwd_ms, 4),
             "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
-            "kernel_ms": {"k_fwd_tc": round(fwd_kms, 4), "k_bwd_tc": round(bwd_kms, 4)},
-            "kernel_tflops": {"k_fwd_tc": round(fwd_ktf, 2), "k_bwd_tc": round(bwd_ktf, 2)},
+            "kernel_ms": {"k_fwd_tc": round(fwd_kms, 4), bwd_name: round(bwd_kms, 4)},
+            "kernel_tflops": {"k_fwd_tc": round(fwd_ktf, 2), bwd_name: round(bwd_ktf, 2)},
             "pct_of_peak": round(100 * value / world / peak, 2),
-            "roofline": {"bound": "tensor", "kernel": f"k_{dominant}_tc",
+            "roofline": {"bound": "tensor", "kernel": bwd_name if dominant == "bwd" else "k_fwd_tc",
                          "units": f"{10 if dominant == 'bwd' else 4}*D*kept_pairs FLOPs per launch",
                          "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
                          "frac": round(achieved / peak, 4), "peak_source": f"{which} bf16 burst",
@@ -401,7 +408,7 @@ def run_ours(args):
             "e2e": {"value": round(job_tflops(world, step_flops, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": LAUNCHES_PER_STEP * args.steps,
+            "gpu_launches": (LAUNCHES_PER_STEP_DET if args.deterministic else LAUNCHES_PER_STEP) * args.steps,
             "status_flags": flags,
             "clocks": clk.summary(),
         }
@@ -436,6 +443,8 @@ def main():
                     help="smaller batch for C3/C4 (profiler captures only; not a bench line)")
     ap.add_argument("--causal", action="store_true",
                     help="C3 with the causal mask and its lower-triangular block index")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="the deterministic backward (bitwise reproducible dq)")
     args = ap.parse_args()
     if args.causal and args.config != 3:
         ap.error("--causal applies to C3")

@@ -46,7 +46,8 @@ class bsa_params(ctypes.Structure):
     _fields_ = [("q_layout", ctypes.c_int32), ("kv_layout", ctypes.c_int32),
                 ("num_heads", ctypes.c_int64), ("num_kv_heads", ctypes.c_int64),
                 ("block_shape", ctypes.c_int64 * 2), ("scale", ctypes.c_double),
-                ("return_lse", ctypes.c_int32), ("mask_type", ctypes.c_int32)]
+                ("return_lse", ctypes.c_int32), ("mask_type", ctypes.c_int32),
+                ("deterministic", ctypes.c_int32)]
 
 
 class bsa_ws_region(ctypes.Structure):
@@ -112,6 +113,7 @@ class Params:
     scale: float = 0.0
     return_lse: bool = True
     causal: bool = False
+    deterministic: bool = False
 
     def c(self) -> bsa_params:
         p = bsa_params()
@@ -121,6 +123,7 @@ class Params:
         p.scale = float(self.scale)
         p.return_lse = 1 if self.return_lse else 0
         p.mask_type = 1 if self.causal else 0
+        p.deterministic = 1 if self.deterministic else 0
         return p
 
 
@@ -174,10 +177,10 @@ def _stream(stream) -> Optional[int]:
 
 
 def params_for(q_layout, kv_layout, num_heads, num_kv_heads=0, block_shape=(128, 128), scale=0.0,
-               return_lse=True, causal=False) -> Params:
+               return_lse=True, causal=False, deterministic=False) -> Params:
     return Params(q_layout, kv_layout, int(num_heads), int(num_kv_heads),
                   (int(block_shape[0]), int(block_shape[1])), float(scale), bool(return_lse),
-                  bool(causal))
+                  bool(causal), bool(deterministic))
 
 
 def _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table, out, lse):

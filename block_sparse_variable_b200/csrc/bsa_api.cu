@@ -233,6 +233,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   p.scale_log2 = float(scale * 1.4426950408889634);
   p.return_lse = want_lse ? 1 : 0;
   p.causal = P.mask_type == BSA_MASK_CAUSAL ? 1 : 0;
+  p.deterministic = a.bwd && P.deterministic ? 1 : 0;
   p.fwd_slots = fwd_slots; p.bwd_slots = bwd_slots;
   p.fwd_slots_pad = fpad; p.bwd_slots_pad = bpad;
 
@@ -277,12 +278,12 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   place(cur, uint64_t(tk_max) * 4, L.kb_batch);
   place(cur, uint64_t(Hidx) * Rg * W * 2, W_.comp);
   place(cur, uint64_t(Hidx) * Rg * 4, W_.ncomp);
-  const int64_t kpad = a.bwd ? bpad : fpad;
+  // the deterministic backward sorts both work lists through the key buffers
+  const int64_t kpad = !a.bwd ? fpad : p.deterministic ? (fpad > bpad ? fpad : bpad) : bpad;
   place(cur, uint64_t(kpad) * 8, W_.sort_keys);
   place(cur, uint64_t(kpad) * 8, L.sorted);
-  if (!a.bwd) {
-    place(cur, uint64_t(fwd_slots) * 4, W_.fwd_items);
-  } else {
+  if (!a.bwd || p.deterministic) place(cur, uint64_t(fwd_slots) * 4, W_.fwd_items);
+  if (a.bwd) {
     const int64_t nnz_max = Hidx * Rg * (W < tk_max ? W : tk_max);
     place(cur, uint64_t(Hidx) * tk_max * 4, L.inv_cnt);
     place(cur, uint64_t(Hidx) * tk_max * 4, L.inv_sub);
@@ -290,7 +291,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
     place(cur, uint64_t(nnz_max) * 4, W_.inv_list);
     place(cur, uint64_t(bwd_slots) * 4, W_.bwd_items);
     place(cur, uint64_t(rows_q) * N1 * 4, W_.dsum);
-    place(cur, uint64_t(rows_q) * N1 * D * 4, W_.dq_acc);
+    if (!p.deterministic) place(cur, uint64_t(rows_q) * N1 * D * 4, W_.dq_acc);
   }
   W_.Rg = Rg;
   W_.tk_max = tk_max;
@@ -356,12 +357,16 @@ bsa_status run_fwd(const Problem &p, cudaStream_t s, cudaEvent_t e0, cudaEvent_t
 
 bsa_status run_bwd(const Problem &p, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   BSA_LAUNCH(bsa::launch_prep_geometry(p, s));
-  BSA_LAUNCH(bsa::launch_prep_compact(p, false, s));
+  // deterministic: the forward work list too (for the q-major dQ pass),
+  // sorted before the backward keys reuse the key buffers
+  BSA_LAUNCH(bsa::launch_prep_compact(p, p.deterministic != 0, s));
+  if (p.deterministic) BSA_LAUNCH(bsa::launch_sort_items(p, p.fwd_slots_pad, p.fwd_items, s));
   BSA_LAUNCH(bsa::launch_prep_inverse(p, s));
   BSA_LAUNCH(bsa::launch_sort_items(p, p.bwd_slots_pad, p.bwd_items, s));
   BSA_LAUNCH(bsa::launch_bwd_pre(p, s));
   if (e0) BSA_LAUNCH(cudaEventRecord(e0, s));
   BSA_LAUNCH(bsa::launch_bwd_main(p, s));
+  if (p.deterministic) BSA_LAUNCH(bsa::launch_dq_main(p, s));  // inside the events: both main kernels
   if (e1) BSA_LAUNCH(cudaEventRecord(e1, s));
   BSA_LAUNCH(bsa::launch_bwd_post(p, s));
   return BSA_OK;
@@ -398,7 +403,7 @@ bsa_status bsa_set_main_kernel_events(void *before, void *after) {
   return BSA_OK;
 }
 
-int32_t bsa_abi_version(void) { return 2; }
+int32_t bsa_abi_version(void) { return 3; }
 
 const char *bsa_status_string(bsa_status s) {
   switch (s) {

@@ -48,6 +48,7 @@ struct Problem {
   float scale, scale_log2;  // scale, scale * log2(e)
   int32_t return_lse;
   int32_t causal;  // kv token u visible to query row t iff u <= t + kvlen - qlen
+  int32_t deterministic;  // backward: dQ from the q-major pass, no accumulator
 
   // ---- tensors (strides in elements).  Token row t of batch b, head h:
   //   base + b*sb + (tok0_b + t)*st + h*sh   (tok0 = 0 for BNSD, cu[b] for TND)
@@ -82,7 +83,7 @@ struct Problem {
   int32_t *inv_list;    // [nnz_max]
   int32_t *bwd_items;   // [N2*tk_max*ksl]
   float *dsum;          // [rows_q][N1] rowsum(dOut o out)
-  float *dq_acc;        // [rows_q][N1][D]
+  float *dq_acc;        // [rows_q][N1][D]; absent in the deterministic backward
   int64_t fwd_slots, bwd_slots, fwd_slots_pad, bwd_slots_pad;
 };
 
@@ -95,6 +96,7 @@ cudaError_t launch_fwd_main(const Problem &p, cudaStream_t s);
 cudaError_t launch_bwd_pre(const Problem &p, cudaStream_t s);
 cudaError_t launch_bwd_main(const Problem &p, cudaStream_t s);
 cudaError_t launch_bwd_post(const Problem &p, cudaStream_t s);
+cudaError_t launch_dq_main(const Problem &p, cudaStream_t s);
 
 int num_sms();
 

@@ -96,8 +96,10 @@ __global__ void k_kv_zero_tail(const Problem p) {
 }  // namespace
 
 cudaError_t launch_bwd_pre(const Problem &p, cudaStream_t s) {
-  cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, size_t(p.rows_q) * p.N1 * p.D * sizeof(float), s);
-  if (e != cudaSuccess) return e;
+  if (p.dq_acc) {  // absent in the deterministic backward (dq written directly)
+    cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, size_t(p.rows_q) * p.N1 * p.D * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
   const int64_t warps = p.rows_q * p.N1;
   const unsigned grid = unsigned((warps * 32 + 255) / 256);
   if (p.dtype == BSA_BF16) k_bwd_pre<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
@@ -110,10 +112,10 @@ cudaError_t launch_bwd_post(const Problem &p, cudaStream_t s) {
   const unsigned grid = unsigned((n8 + 255) / 256);
   const dim3 zgrid(64, unsigned(p.B));
   if (p.dtype == BSA_BF16) {
-    k_dq_convert<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
+    if (p.dq_acc) k_dq_convert<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
     k_kv_zero_tail<__nv_bfloat16><<<zgrid, 256, 0, s>>>(p);
   } else {
-    k_dq_convert<__half><<<grid, 256, 0, s>>>(p);
+    if (p.dq_acc) k_dq_convert<__half><<<grid, 256, 0, s>>>(p);
     k_kv_zero_tail<__half><<<zgrid, 256, 0, s>>>(p);
   }
   return cudaGetLastError();

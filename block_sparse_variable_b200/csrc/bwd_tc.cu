@@ -154,7 +154,7 @@ __device__ __forceinline__ int b_t0(const Problem &p, const BItem &v, const BSte
   return b_qblock(p, v, c.hh, c.e, TK) * p.BQ + c.st * 128;
 }
 
-template <int D, bool BF16, bool kCausal>
+template <int D, bool BF16, bool kCausal, bool kDQ>
 __global__ void __launch_bounds__(kBThreads, 1)
     k_bwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
@@ -184,7 +184,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kBarKVEmpty), 1);
     for (int s = 0; s < 2; ++s) {
       mbar_init(bar(kBarQD + s), 1);
-      mbar_init(bar(kBarDQOut + s), 256);
+      // with dQ: the softmax warps' 256 arrivals once the step's dQ is staged;
+      // without: the MMA issuer's commit once the step's MMAs are done
+      mbar_init(bar(kBarDQOut + s), kDQ ? 256 : 1);
     }
     mbar_init(bar(kBarS), 1);
     mbar_init(bar(kBarDS), 256);
@@ -224,12 +226,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
     // memory; the additions into global memory then proceed on their own.
     // One commit group per tile: the Q tile's boxes, then the dOut tile's.
     auto reduce_slot = [&](int sl) {
+      if constexpr (kDQ) {
 #pragma unroll
-      for (int j = 0; j < D / 32; ++j) {
-        const uint32_t src = j < D / 64 ? sQ + sl * L::kTile + j * L::kBox
-                                        : sDO + sl * L::kTile + (j - D / 64) * L::kBox;
-        tma_reduce_add_3d(&map_dq, src, 32 * j, pend_h[sl], pend_row[sl]);
-        if (j == D / 64 - 1 || j == D / 32 - 1) bulk_commit();
+        for (int j = 0; j < D / 32; ++j) {
+          const uint32_t src = j < D / 64 ? sQ + sl * L::kTile + j * L::kBox
+                                          : sDO + sl * L::kTile + (j - D / 64) * L::kBox;
+          tma_reduce_add_3d(&map_dq, src, 32 * j, pend_h[sl], pend_row[sl]);
+          if (j == D / 64 - 1 || j == D / 32 - 1) bulk_commit();
+        }
       }
     };
     auto flush = [&](uint32_t s) -> bool {  // the last two steps, after the loop
@@ -287,14 +291,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         __syncwarp();
         if (lane == 0) {
-          if (refill) reduce_slot(slot);
+          if (kDQ && refill) reduce_slot(slot);
           mbar_expect_tx(bar(kBarQD + slot), 2 * L::kTile);
           armed_qd[slot] = int((sk >> 1) & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
-          if (refill) bulk_wait_read<1>();
+          if (kDQ && refill) bulk_wait_read<1>();
           tma_load_5d(sQ + slot * L::kTile, &map_q, bar(kBarQD + slot), 0, tok, 0, h1, bb);
-          if (refill) bulk_wait_read<0>();
+          if (kDQ && refill) bulk_wait_read<0>();
           tma_load_5d(sDO + slot * L::kTile, &map_do, bar(kBarQD + slot), 0, tok, 0, h1, bb);
         }
         __syncwarp();
@@ -303,13 +307,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
         ++sk;
       }
     }
-    for (uint32_t s = sk >= 2 ? sk - 2 : 0; s < sk && ok; ++s) ok = flush(s);
+    if (kDQ)
+      for (uint32_t s = sk >= 2 ? sk - 2 : 0; s < sk && ok; ++s) ok = flush(s);
     if (*abort && lane == 0) {  // let every copy already issued land before the CTA exits
       if (armed_kv >= 0) drain_wait(bar(kBarKV), uint32_t(armed_kv));
       for (int s = 0; s < 2; ++s)
         if (armed_qd[s] >= 0) drain_wait(bar(kBarQD + s), uint32_t(armed_qd[s]));
     }
-    if (lane == 0) bulk_wait_all();  // every dQ addition has been made
+    if (kDQ && lane == 0) bulk_wait_all();  // every dQ addition has been made
   } else if (warp == kBMmaWarp) {
     // ------------------------------------------------------- MMA issuer
     constexpr uint32_t idSP = idesc_f16(BF16, 128, 128, false, false);  // S^T, dP^T
@@ -360,7 +365,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
         }
         __syncwarp();
         // R1 still holds the previous step's dQ until it has been read out
-        if (sk > 0 && !(ok = wait_warp(bar(kBarDQOut + ((sk - 1) & 1u)), ((sk - 1) >> 1) & 1u, abort, p.status)))
+        // (without dQ it held dP^T, read before the previous step's dS_full)
+        if (kDQ && sk > 0 &&
+            !(ok = wait_warp(bar(kBarDQOut + ((sk - 1) & 1u)), ((sk - 1) >> 1) & 1u, abort, p.status)))
           break;
         tc_fence_after();
         if (lane == 0) {
@@ -381,9 +388,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const uint32_t acc = (first && kk == 0) ? 0u : 1u;
             mma_ts(tdV, tR0 + pcol, dOmn + uint64_t(kk * 128), idKV, acc);
             mma_ts(tdK, tR0 + 32u + pcol, dQmn + uint64_t(kk * 128), idKV, acc);
-            mma_ss(tR1, dDS + uint64_t(kk * 128), dKmn + uint64_t(kk * 128), idQ, kk > 0 ? 1u : 0u);
+            if constexpr (kDQ) mma_ss(tR1, dDS + uint64_t(kk * 128), dKmn + uint64_t(kk * 128), idQ, kk > 0 ? 1u : 0u);
           }
           mma_commit(bar(kBarP2));
+          if constexpr (!kDQ) mma_commit(bar(kBarDQOut + slot));  // the slot's Q, dOut are free
         }
         __syncwarp();
         first = false;
@@ -472,7 +480,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
         // them as S), dS also into shared memory for the dQ product
         tmem_st32(tR0 + lane_off + uint32_t(64 * wg), pp);
         tmem_st32(tR0 + lane_off + uint32_t(64 * wg + 32), dd);
-        {
+        if constexpr (kDQ) {
           // dS^T row r, q columns [64w, 64w+64): one 128-byte swizzled row
           uint4 *row = reinterpret_cast<uint4 *>(sbase + L::kDS + wg * L::kBox + r * 128);
 #pragma unroll
@@ -480,9 +488,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
             row[c ^ (r & 7)] = make_uint4(dd[4 * c], dd[4 * c + 1], dd[4 * c + 2], dd[4 * c + 3]);
         }
         tmem_wait_st();
-        fence_proxy_async_smem();
+        if constexpr (kDQ) fence_proxy_async_smem();
         tc_fence_before();
         mbar_arrive(bar(kBarDS));
+        if constexpr (!kDQ) {  // dQ comes from the q-major pass
+          ++sk;
+          ++nsteps;
+          continue;
+        }
         // dQ of the step (TMEM lanes = q rows) out to shared memory, where the
         // step's Q and dOut tiles were (free once its MMAs are done): four
         // boxes of 32 fp32 columns x 128 rows in the 128-byte swizzle, group
@@ -568,15 +581,24 @@ __global__ void __launch_bounds__(kBThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool kCausal>
+template <int D, bool BF16, bool kCausal, bool kDQ>
 cudaError_t launch_bwd_tc(const Problem &p, const BwdMaps &m, cudaStream_t s) {
   const int smem = BLayout<D>::kBytes > 120 * 1024 ? BLayout<D>::kBytes : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<D, BF16, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(k_bwd_tc<D, BF16, kCausal, kDQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.bwd_slots < num_sms() ? p.bwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_bwd_tc<D, BF16, kCausal><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
+  k_bwd_tc<D, BF16, kCausal, kDQ><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
   return cudaGetLastError();
+}
+
+// the causal mask and the deterministic mode (dQ left to the q-major pass)
+// are separate instantiations: the plain kernel carries neither
+template <bool kCausal, bool kDQ>
+cudaError_t launch_bwd_for(const Problem &p, const BwdMaps &m, cudaStream_t s) {
+  if (p.dtype == BSA_BF16)
+    return p.D == 64 ? launch_bwd_tc<64, true, kCausal, kDQ>(p, m, s) : launch_bwd_tc<128, true, kCausal, kDQ>(p, m, s);
+  return p.D == 64 ? launch_bwd_tc<64, false, kCausal, kDQ>(p, m, s) : launch_bwd_tc<128, false, kCausal, kDQ>(p, m, s);
 }
 
 }  // namespace
@@ -585,16 +607,9 @@ cudaError_t launch_bwd_main(const Problem &p, cudaStream_t s) {
   BwdMaps m;
   cudaError_t e = make_bwd_maps(p, m);
   if (e != cudaSuccess) return e;
-  // the causal mask is a separate instantiation: the unmasked kernel carries
-  // none of its arithmetic
-  if (p.causal) {
-    if (p.dtype == BSA_BF16)
-      return p.D == 64 ? launch_bwd_tc<64, true, true>(p, m, s) : launch_bwd_tc<128, true, true>(p, m, s);
-    return p.D == 64 ? launch_bwd_tc<64, false, true>(p, m, s) : launch_bwd_tc<128, false, true>(p, m, s);
-  }
-  if (p.dtype == BSA_BF16)
-    return p.D == 64 ? launch_bwd_tc<64, true, false>(p, m, s) : launch_bwd_tc<128, true, false>(p, m, s);
-  return p.D == 64 ? launch_bwd_tc<64, false, false>(p, m, s) : launch_bwd_tc<128, false, false>(p, m, s);
+  if (p.deterministic)
+    return p.causal ? launch_bwd_for<true, false>(p, m, s) : launch_bwd_for<false, false>(p, m, s);
+  return p.causal ? launch_bwd_for<true, true>(p, m, s) : launch_bwd_for<false, true>(p, m, s);
 }
 
 }  // namespace bsa

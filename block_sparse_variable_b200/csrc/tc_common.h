@@ -29,4 +29,12 @@ struct BwdMaps {
 
 cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m);
 
+// the q-major dQ pass of the deterministic backward streams Q and dOut with
+// the q-tensor box and K, V with the kv box
+struct DqMaps {
+  CUtensorMap q, k, v, dout;
+};
+
+cudaError_t make_dq_maps(const Problem &p, DqMaps &m);
+
 }  // namespace bsa

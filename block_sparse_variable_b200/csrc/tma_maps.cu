@@ -2,6 +2,7 @@
 // driver's cuTensorMapEncodeTiled is reached through the runtime's
 // entry-point query, so the library needs no link-time libcuda.
 #include <cuda.h>
+#include <cstring>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -106,7 +107,19 @@ cudaError_t make_bwd_maps(const Problem &p, BwdMaps &m) {
   if ((e = q_map(&m.dout, p, p.dout, p.do_sb, p.do_sh, p.do_st)) != cudaSuccess) return e;
   if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
   if ((e = kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st)) != cudaSuccess) return e;
+  if (!p.dq_acc) {  // deterministic backward: no accumulator, the map is never used
+    std::memset(&m.dq_acc, 0, sizeof(m.dq_acc));
+    return cudaSuccess;
+  }
   return dq_acc_map(&m.dq_acc, p);
+}
+
+cudaError_t make_dq_maps(const Problem &p, DqMaps &m) {
+  cudaError_t e = q_map(&m.q, p, p.q, p.q_sb, p.q_sh, p.q_st);
+  if (e != cudaSuccess) return e;
+  if ((e = q_map(&m.dout, p, p.dout, p.do_sb, p.do_sh, p.do_st)) != cudaSuccess) return e;
+  if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
+  return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);
 }
 
 }  // namespace bsa

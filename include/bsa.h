@@ -86,6 +86,8 @@ typedef struct bsa_params {
   double scale;           /* 0 means 1/sqrt(D) */
   int32_t return_lse;     /* forward only: write lse when non-zero */
   int32_t mask_type;      /* BSA_MASK_NONE or BSA_MASK_CAUSAL */
+  int32_t deterministic;  /* backward only: non-zero for bitwise reproducible
+                             dq (see bsa_bwd); forward: ignored */
 } bsa_params;
 
 /* Token mask inside the selected blocks (GenericBlockSparseAttention article,
@@ -189,6 +191,15 @@ bsa_status bsa_fwd_static_workspace(const bsa_tensor *q, const bsa_tensor *k, co
  *             written (zeros where no query selects it), except that under
  *             PA_BBND only the pages block_table[b][0 .. ceil(kvlen_b/page))
  *             are written; other pages are left untouched.
+ * By default dq is summed in fp32 from many CTAs through the L2 (order of
+ * the additions varies between runs, so dq may differ in its last bits).
+ * With params->deterministic set, dq comes from a separate query-major pass
+ * that recomputes P and dS and sums each row's contributions in index order
+ * on one SM (the deterministic template of the aclnnFlashAttention-
+ * UnpaddingScoreGradV2 article, section 6.1: no two cores add into the same
+ * address), so dq, dk and dv are bitwise the same on every run; it costs
+ * the q-major pass's extra S and dP products.  The workspace size depends on
+ * the flag.
  */
 bsa_status bsa_bwd_get_workspace(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
                                  const bsa_tensor *out, const bsa_tensor *dout,
@@ -265,8 +276,9 @@ bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, co
 /* Profiling hook (the pages have no counterpart).  The next bsa_fwd or
  * bsa_bwd call made by this host thread records `before` and `after`
  * (cudaEvent_t handles created by the caller, passed as void*) on its stream
- * immediately before and after its main attention kernel, so that kernel's
- * duration can be timed apart from the preparation kernels; the setting is
+ * immediately before and after its main attention kernel (the deterministic
+ * backward: its two main kernels, kv-major dK/dV and q-major dQ), so that
+ * kernel's duration can be timed apart from the preparation kernels; the setting is
  * then cleared, whatever the call's outcome: a call that launches nothing
  * (failed validation, an empty problem) records nothing.  Both NULL clears a
  * pending pair; exactly one NULL returns BSA_ERR_NULLPTR.  bsa_fwd_static_
@@ -291,7 +303,7 @@ bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64
 bsa_status bsa_selftest_wait_timeout(uint32_t *flags, void *stream);
 
 /* Library ABI version (bumped on any signature or layout change; 2 added
- * bsa_params.mask_type). */
+ * bsa_params.mask_type, 3 bsa_params.deterministic). */
 int32_t bsa_abi_version(void);
 
 #ifdef __cplusplus

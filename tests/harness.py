@@ -19,7 +19,7 @@ LSE_ABS = 1e-3
 
 def params_of(p, return_lse=True) -> bsa.Params:
     return bsa.params_for(p.layout_q, p.layout_kv, p.N1, p.N2, (p.BQ, p.BKV), p.scale, return_lse,
-                          getattr(p, "causal", False))
+                          getattr(p, "causal", False), getattr(p, "deterministic", False))
 
 
 def device_inputs(p, device="cuda"):

@@ -25,7 +25,7 @@ def test_exports_every_declared_symbol():
     for n in names:
         assert hasattr(bsa.lib(), n), n
     assert set(names) == set(bsa.EXPORTED)
-    assert bsa.lib().bsa_abi_version() == 2
+    assert bsa.lib().bsa_abi_version() == 3
 
 
 def test_status_strings():
@@ -169,3 +169,22 @@ def test_mask_type_must_be_known():
     bad = Bad(**{f.name: getattr(P, f.name) for f in dataclasses.fields(P)})
     assert _code(lambda: _ws(p, params=bad)) == 161002
     assert _ws(p, params=dataclasses.replace(P, causal=True)) == _ws(p)
+
+
+def test_deterministic_backward_workspace():
+    """The deterministic backward holds the forward work list and no dQ
+    accumulator; the forward ignores the flag."""
+    import dataclasses
+    p = _prob()
+    P = params_of(p)
+    Pd = dataclasses.replace(P, deterministic=True)
+    lse = torch.empty(p.q.shape[0], p.N1)
+    kw = dict(cu_seqlens_q=p.cu_q, cu_seqlens_kv=p.cu_kv)
+    lay = bsa.bsa_bwd_workspace_layout(p.q, p.k, p.v, p.q, p.dout, lse, p.index, P, **kw)
+    lay_d = bsa.bsa_bwd_workspace_layout(p.q, p.k, p.v, p.q, p.dout, lse, p.index, Pd, **kw)
+    assert lay.dq_acc.bytes and not lay.fwd_items.bytes
+    assert lay_d.fwd_items.bytes and not lay_d.dq_acc.bytes
+    assert lay_d.sort_keys.bytes >= lay.sort_keys.bytes
+    assert bsa.bsa_bwd_get_workspace(p.q, p.k, p.v, p.q, p.dout, lse, p.index, Pd, **kw) \
+        == lay_d.total_bytes
+    assert _ws(p, params=Pd) == _ws(p)

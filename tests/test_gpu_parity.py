@@ -185,6 +185,55 @@ def test_causal_cases(name):
     _run_and_check(p)
 
 
+# deterministic backward: dK/dV from the kv-major kernel without its dQ
+# reductions, dQ from the q-major pass; parity as above, the forward work
+# list in the backward workspace exact, and a second call bitwise identical
+DETERMINISTIC = ["bnsd_random", "bnsd_ragged_kv", "bnsd_blocks_256x128", "bnsd_fp16_d128",
+                 "tnd_gqa", "tnd_shared_rows", "tnd_seqused", "tnd_empty_batches", "paged",
+                 "paged_256", "big_blocks", "blocks_1024", "dense_many_blocks", "invalid_entries",
+                 "empty_rows", "causal_tnd_q_longer", "causal_paged", "causal_bnsd_128x512"]
+
+
+def _check_deterministic(p):
+    p.deterministic = True
+    _run_and_check(p)
+    R = _oracle(p)
+    d = H.device_inputs(p)
+    out_b, lse_f = R["out_b"].cuda(), R["lse_f"].cuda()
+    first = H.gpu_bwd(p, out_b, lse_f, d)
+    second = H.gpu_bwd(p, out_b, lse_f, d)
+    torch.cuda.synchronize()
+    wm = H.kv_written_mask(p).cuda()  # paged: pages the call does not own stay untouched
+    for name, a, b in zip(("dq", "dk", "dv"), first[:3], second[:3]):
+        if name != "dq":
+            a, b = a[wm], b[wm]
+        assert torch.equal(a.view(torch.int16), b.view(torch.int16)), f"{name} differs between runs"
+    ws_b = first[3]
+    lay_b = bsa.bsa_bwd_workspace_layout(d["q"], d["k"], d["v"], out_b, d["dout"], lse_f, d["index"],
+                                         H.params_of(p), **H.opt_kwargs(d))
+    assert lay_b.dq_acc.bytes == 0 and lay_b.fwd_items.bytes > 0
+    st = H.region(ws_b, lay_b.status, torch.int32)
+    B = builders.build_all(p)
+    n_f = int(st[2])
+    assert n_f == len(B["fwd_items"])
+    assert np.array_equal(H.region(ws_b, lay_b.fwd_items, torch.int32, n_f), B["fwd_items"])
+
+
+@pytest.mark.parametrize("name", DETERMINISTIC)
+def test_deterministic_backward(name):
+    _check_deterministic(_problem(name))
+
+
+@pytest.mark.parametrize("name", ["tnd_seqused", "paged_256"])
+def test_deterministic_backward_nan_in_unused_kv(name):
+    _check_deterministic(_poison_unused_kv(_problem(name)))
+
+
+@pytest.mark.parametrize("c", [1, 2])
+def test_deterministic_backward_configs(c):
+    _check_deterministic(workloads.make_config(c))
+
+
 def _poison_unused_kv(p):
     """NaN in every stored K/V row the attention must not use: rows past
     seqused_kv (BNSD, TND), the tail of each last page and whole unused pages
