@@ -100,3 +100,50 @@ def kv_written_mask(p) -> torch.Tensor:
         for x in range(n):
             m[int(p.block_table[b, x])] = True
     return m
+
+
+# ---------------------------------------------------------------- FP8 inputs
+E4M3_HALF_ULP_REL = 2.0 ** -4   # 3 mantissa bits: round to nearest within 2^-4 relative
+E4M3_HALF_SUB = 2.0 ** -10      # half the subnormal spacing 2^-9
+
+
+def fp8_out_bound(p) -> torch.Tensor:
+    """Element bound on |out - exact out| when P is cast to e4m3 before P V.
+
+    The kernel computes P against a reference m no larger than the row max
+    and sums l from the unrounded fp32 P, so with P_u = exp(s_u - max) and
+    L = sum_u P_u (both exact, fp64), the cast changes out_d by at most
+    sum_u (2^-4 P_u + 2^-10) |v_ud| / L: a relative 2^-4 for normal e4m3
+    values, an absolute 2^-10 (scaled down by the later rescale, never up)
+    below them.  Built from torch library routines on the dense token mask;
+    a row that sees nothing has bound 0 (its out must be exactly 0)."""
+    from tests import torch_reference as TR
+    q, k, v = p.q.double(), p.k.double(), p.v.double()
+    g = p.N1 // p.N2
+    per = []
+    for b in range(p.B):
+        qb, kb, vb = TR.batch_tensors(p, b, q, k, v)
+        kb, vb = kb.repeat_interleave(g, 0), vb.repeat_interleave(g, 0)
+        mask = TR.token_mask(p, b)
+        s = (p.scale * torch.matmul(qb, kb.transpose(-1, -2))).masked_fill(~mask, float("-inf"))
+        m = s.amax(-1, keepdim=True)
+        m = torch.where(torch.isfinite(m), m, torch.zeros_like(m))
+        pr = torch.exp(s - m) * mask
+        L = pr.sum(-1, keepdim=True)
+        num = torch.matmul(E4M3_HALF_ULP_REL * pr + E4M3_HALF_SUB * mask.double(), vb.abs())
+        per.append((torch.where(L > 0, num / L.clamp(min=1e-300), torch.zeros_like(num)), None))
+    return TR.to_q_layout(p, per, 0)
+
+
+def check_fp8_out(got: torch.Tensor, ref: torch.Tensor, bound: torch.Tensor, odtype):
+    """Every element within the P-cast bound plus the output's own rounding
+    (half an ulp of the output dtype) and a 1e-5 allowance for the fp32
+    accumulation and exp2 approximation."""
+    g, r, bd = got.double().cpu(), ref.double().cpu(), bound.double().cpu()
+    assert torch.isfinite(g).all(), "out: non-finite values"
+    half_ulp = 2.0 ** -9 if odtype == torch.bfloat16 else 2.0 ** -12
+    lim = bd + half_ulp * r.abs() + 1e-5
+    excess = float(((g - r).abs() - lim).max()) if g.numel() else -1.0
+    assert excess <= 0, f"out: exceeds the e4m3 P-cast bound by {excess:.3e}"
+    used = float(((g - r).abs() / lim).max()) if g.numel() else 0.0
+    return used

@@ -50,6 +50,12 @@ class Problem:
     lens_q: List[int] = field(default_factory=list)
     lens_kv: List[int] = field(default_factory=list)
     causal: bool = False     # kv token u visible to query row t iff u <= t + kvlen - qlen
+    out_dtype: Optional[torch.dtype] = None  # out / dout dtype when q, k, v are 8-bit
+
+    @property
+    def odtype(self) -> torch.dtype:
+        """dtype of out (and dout): the input dtype, or out_dtype for FP8 inputs."""
+        return self.out_dtype if self.out_dtype is not None else self.dtype
 
     @property
     def W(self) -> int:
@@ -152,7 +158,8 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
                  Sq=None, Skv=None, kv_storage=None, Hidx=None, W=None,
                  pattern: Callable = pat_random_k, page_size=128, extra_pages=0,
                  use_seqused_kv=None, seed_base=0, scale=None, max_pages=None,
-                 row_hook: Optional[Callable] = None, causal: bool = False) -> Problem:
+                 row_hook: Optional[Callable] = None, causal: bool = False,
+                 out_dtype: Optional[torch.dtype] = None) -> Problem:
     """Build one seeded problem.
 
     lens_q / lens_kv: per-batch valid lengths (TND q: the stored lengths).
@@ -161,7 +168,13 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
     seqused_kv carries the used lengths).
     row_hook(rng, b, hi, i, row_list) -> list[int]: lets a test write raw
     slot values (0xFFFF in mid-row, out-of-range or repeated ids).
+    dtype torch.float8_e4m3fn: q, k, v are N(0,1) rounded to e4m3 (the
+    GenericBlockSparseAttention FP8 inputs); out_dtype (default bf16) is the
+    dtype of out and dout.
     """
+    if dtype == torch.float8_e4m3fn and out_dtype is None:
+        out_dtype = torch.bfloat16
+    odt = out_dtype if out_dtype is not None else dtype
     s = seed_base
     lens_q = list(lens_q) if lens_q is not None else [Sq] * B
     lens_kv = list(lens_kv) if lens_kv is not None else list(lens_q)
@@ -174,12 +187,12 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
         Sq = Sq if Sq is not None else max(lens_q)
         assert all(l == Sq for l in lens_q), "BNSD query rows are all valid"
         q = _randn((B, N1, Sq, D), s + 1, dtype)
-        dout = _randn((B, N1, Sq, D), s + 4, dtype)
+        dout = _randn((B, N1, Sq, D), s + 4, odt)
     else:
         Tq = sum(lens_q)
         cu_q = torch.tensor([0] + list(np.cumsum(lens_q)), dtype=torch.int64)
         q = _randn((Tq, N1, D), s + 1, dtype)
-        dout = _randn((Tq, N1, D), s + 4, dtype)
+        dout = _randn((Tq, N1, D), s + 4, odt)
 
     if layout_kv == "BNSD":
         Skv = Skv if Skv is not None else max(lens_kv)
@@ -240,7 +253,7 @@ def make_problem(*, name="custom", layout_q="BNSD", layout_kv="BNSD", B=1, N1=2,
                    dtype=dtype, BQ=BQ, BKV=BKV, Hidx=Hidx, scale=scale, q=q, k=k, v=v,
                    dout=dout, index=index, cu_q=cu_q, cu_kv=cu_kv, seqused_kv=seqused,
                    block_table=block_table, page_size=(page_size if layout_kv == "PA_BBND" else 0),
-                   lens_q=lens_q, lens_kv=lens_kv, causal=causal)
+                   lens_q=lens_q, lens_kv=lens_kv, causal=causal, out_dtype=out_dtype)
 
 
 # ----------------------------------------------------------------------------
