@@ -20,7 +20,7 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsa.so")
 
-BSA_F16, BSA_BF16, BSA_F32, BSA_U16, BSA_I32, BSA_I64 = 1, 2, 3, 4, 5, 6
+BSA_F16, BSA_BF16, BSA_F32, BSA_U16, BSA_I32, BSA_I64, BSA_F8E4M3 = 1, 2, 3, 4, 5, 6, 7
 LAYOUTS = {"BNSD": 0, "TND": 1, "PA_BBND": 2}
 FLAG_BAD_INDEX, FLAG_BAD_SEQLEN, FLAG_BAD_PAGE, FLAG_TIMEOUT = 1, 2, 4, 8
 STATUS_NAMES = {0: "BSA_OK", 161001: "BSA_ERR_NULLPTR", 161002: "BSA_ERR_PARAM_INVALID",
@@ -28,7 +28,8 @@ STATUS_NAMES = {0: "BSA_OK", 161001: "BSA_ERR_NULLPTR", 161002: "BSA_ERR_PARAM_I
                 561000: "BSA_ERR_CUDA", 561103: "BSA_ERR_INNER"}
 
 _DTYPES = {torch.float16: BSA_F16, torch.bfloat16: BSA_BF16, torch.float32: BSA_F32,
-           torch.uint16: BSA_U16, torch.int32: BSA_I32, torch.int64: BSA_I64}
+           torch.uint16: BSA_U16, torch.int32: BSA_I32, torch.int64: BSA_I64,
+           torch.float8_e4m3fn: BSA_F8E4M3}
 
 
 class BsaError(RuntimeError):
@@ -83,10 +84,12 @@ def _load():
     lib.bsa_abi_version.restype = ctypes.c_int32
     lib.bsa_set_main_kernel_events.argtypes = [vp, vp]
     lib.bsa_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
+    lib.bsa_selftest_e4m3.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.bsa_selftest_wait_timeout.argtypes = [vp, vp]
     for f in ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_fwd_workspace_layout",
               "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status",
-              "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout"):
+              "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout",
+              "bsa_selftest_e4m3"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -96,7 +99,8 @@ _lib = _load()
 EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bwd",
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
             "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace",
-            "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout")
+            "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout",
+            "bsa_selftest_e4m3")
 
 
 def lib():
@@ -224,8 +228,8 @@ def bsa_fwd_workspace_layout(q, k, v, index, params: Params, *, cu_seqlens_q=Non
 def bsa_fwd(q, k, v, index, params: Params, *, cu_seqlens_q=None, cu_seqlens_kv=None,
             seqused_kv=None, block_table=None, out=None, lse=None, workspace=None, stream=None):
     """Forward pass on the current (or given) stream.  Returns (out, lse, workspace)."""
-    if out is None:
-        out = torch.empty_like(q)
+    if out is None:  # e4m3 inputs: bf16 out unless the caller passes its own
+        out = torch.empty_like(q, dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype)
     if lse is None and params.return_lse:
         lse = torch.empty(_lse_shape(q, params), dtype=torch.float32, device=q.device)
     ins, o, l = _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table,
@@ -320,6 +324,16 @@ def bsa_selftest_exp2(x: torch.Tensor, stream=None):
     return yp, ym
 
 
+def bsa_selftest_e4m3(x: torch.Tensor, stream=None) -> torch.Tensor:
+    """Pack a CUDA float32 tensor (numel % 4 == 0) into e4m3 bytes with the
+    FP8 forward's routine; returns a uint8 tensor of the same numel."""
+    x = x.contiguous()
+    y = torch.empty(x.numel() // 4, dtype=torch.int32, device=x.device)
+    _check(_lib.bsa_selftest_e4m3(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()),
+                                  x.numel(), ctypes.c_void_p(_stream(stream))), "bsa_selftest_e4m3")
+    return y.view(torch.uint8)
+
+
 def bsa_selftest_wait_timeout(flags: torch.Tensor, stream=None):
     """Run the bounded-wait self test; `flags` is a zeroed int32 CUDA tensor
     whose word 0 receives BSA_FLAG_TIMEOUT."""
@@ -357,8 +371,8 @@ def bsa_fwd_static_workspace(q, k, v, index, params: Params, *, cu_seqlens_q=Non
         T = ctypes.POINTER(bsa_tensor)
         f.argtypes = [T] * 8 + [ctypes.POINTER(bsa_params), T, T, ctypes.c_void_p]
         f.restype = ctypes.c_int
-    if out is None:
-        out = torch.empty_like(q)
+    if out is None:  # e4m3 inputs: bf16 out unless the caller passes its own
+        out = torch.empty_like(q, dtype=torch.bfloat16 if q.dtype == torch.float8_e4m3fn else q.dtype)
     if lse is None and params.return_lse:
         lse = torch.empty(_lse_shape(q, params), dtype=torch.float32, device=q.device)
     ins, o, l = _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table,

@@ -44,14 +44,16 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 bool block_ok(int64_t x) { return x == 128 || x == 256 || x == 512 || x == 1024; }
 
 // A dense-value tensor (q/k/v/out/...): given ndim, dtype, last stride 1, the
-// other strides multiples of 8 elements and a 16-byte-aligned base (16-byte
-// vector loads and TMA boxes start on 16-byte boundaries).
+// other strides 16-byte multiples (8 16-bit or 16 8-bit elements) and a
+// 16-byte-aligned base (16-byte vector loads and TMA boxes start on 16-byte
+// boundaries).
 bsa_status check_values(const bsa_tensor *t, int ndim, int dtype) {
   if (t->ndim != ndim || t->dtype != dtype) return BSA_ERR_PARAM_INVALID;
   if (t->stride[ndim - 1] != 1) return BSA_ERR_PARAM_INVALID;
+  const int64_t per16 = dtype == BSA_F8E4M3 ? 16 : 8;
   for (int i = 0; i < ndim; ++i) {
     if (t->shape[i] < 0) return BSA_ERR_PARAM_INVALID;
-    if (i < ndim - 1 && (t->stride[i] % 8 != 0 || t->stride[i] < 0)) return BSA_ERR_PARAM_INVALID;
+    if (i < ndim - 1 && (t->stride[i] % per16 != 0 || t->stride[i] < 0)) return BSA_ERR_PARAM_INVALID;
   }
   if (reinterpret_cast<uintptr_t>(t->data) % 16 != 0) return BSA_ERR_PARAM_INVALID;
   return BSA_OK;
@@ -100,15 +102,22 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
         (ql == BSA_LAYOUT_TND && (kl == BSA_LAYOUT_TND || kl == BSA_LAYOUT_PA_BBND))))
     return BSA_ERR_PARAM_INVALID;
   const int dt = a.q->dtype;
-  if (dt != BSA_F16 && dt != BSA_BF16) return BSA_ERR_PARAM_INVALID;
+  if (dt != BSA_F16 && dt != BSA_BF16 && dt != BSA_F8E4M3) return BSA_ERR_PARAM_INVALID;
+  const bool fp8 = dt == BSA_F8E4M3;
+  if (fp8 && a.bwd) return BSA_ERR_UNSUPPORTED;  // the backward takes 16-bit inputs
+  // FP8 inputs write a 16-bit out whose dtype is the caller's choice
+  const int odt = fp8 ? a.out->dtype : dt;
+  if (odt != BSA_F16 && odt != BSA_BF16) return BSA_ERR_PARAM_INVALID;
   const int qnd = ql == BSA_LAYOUT_BNSD ? 4 : 3;
   const int knd = kl == BSA_LAYOUT_TND ? 3 : 4;
   bsa_status st;
   if ((st = check_values(a.q, qnd, dt)) != BSA_OK) return st;
   if ((st = check_values(a.k, knd, dt)) != BSA_OK) return st;
   if ((st = check_values(a.v, knd, dt)) != BSA_OK) return st;
-  if ((st = check_values(a.out, qnd, dt)) != BSA_OK) return st;
-  if (!same_shape(a.q, a.out) || !same_shape(a.k, a.v)) return BSA_ERR_PARAM_INVALID;
+  if ((st = check_values(a.out, qnd, odt)) != BSA_OK) return st;
+  if (a.out->ndim != a.q->ndim || !same_shape(a.k, a.v)) return BSA_ERR_PARAM_INVALID;
+  for (int i = 0; i < a.q->ndim; ++i)
+    if (a.out->shape[i] != a.q->shape[i]) return BSA_ERR_PARAM_INVALID;
   if (a.bwd) {
     if ((st = check_values(a.dout, qnd, dt)) != BSA_OK) return st;
     if ((st = check_values(a.dq, qnd, dt)) != BSA_OK) return st;
@@ -125,6 +134,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   if (P.num_heads != N1 || N2 <= 0 || N1 % N2 != 0) return BSA_ERR_PARAM_INVALID;
   if (a.k->shape[knd - 1] != D) return BSA_ERR_PARAM_INVALID;
   if (D != 64 && D != 128) return BSA_ERR_UNSUPPORTED;
+  if (fp8 && D != 128) return BSA_ERR_UNSUPPORTED;  // one 128-byte box per row
   const int64_t BQ = P.block_shape[0], BKV = P.block_shape[1];
   if (!block_ok(BQ) || !block_ok(BKV)) return BSA_ERR_PARAM_INVALID;
   if (!(P.scale >= 0.0) || std::isinf(P.scale)) return BSA_ERR_PARAM_INVALID;
@@ -223,7 +233,7 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   p.B = int32_t(B); p.N1 = int32_t(N1); p.N2 = int32_t(N2); p.D = int32_t(D);
   p.g = int32_t(N1 / N2); p.Hidx = int32_t(Hidx); p.BQ = int32_t(BQ); p.BKV = int32_t(BKV);
   p.W = int32_t(W); p.nsub = int32_t(nsub); p.ksl = int32_t(ksl);
-  p.q_layout = ql; p.kv_layout = kl; p.dtype = dt;
+  p.q_layout = ql; p.kv_layout = kl; p.dtype = dt; p.out_dtype = odt;
   p.Sq = Sq; p.Skv = Skv; p.Tq = Tq; p.Tkv = Tkv;
   p.R = int32_t(R); p.Rg = int32_t(Rg); p.tk_max = int32_t(tk_max);
   p.page_size = int32_t(page); p.max_pages = int32_t(max_pages); p.num_pages = int32_t(num_pages);

@@ -39,6 +39,7 @@ struct Problem {
   // ---- sizes
   int32_t B, N1, N2, D, g, Hidx, BQ, BKV, W, nsub, ksl;
   int32_t q_layout, kv_layout, dtype;
+  int32_t out_dtype;  // dtype of out: dtype, or F16 / BF16 for F8E4M3 inputs
   int64_t Sq, Skv, Tq, Tkv;
   int32_t R;        // index rows per (batch, head) for BNSD; total rows for TND
   int32_t Rg;       // global query-block rows

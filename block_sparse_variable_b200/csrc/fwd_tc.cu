@@ -40,6 +40,7 @@
 #include "addr.cuh"
 #include "bsa_internal.h"
 #include "exp2_poly.cuh"
+#include "fp8.cuh"
 #include "fwd_walk.cuh"
 #include "ptx_sm80.cuh"
 #include "sm100.cuh"
@@ -87,10 +88,10 @@ enum : int {
   kNumBars = 31
 };
 
-template <int D>
+template <int D, bool kFp8>
 struct Layout {
-  static constexpr int kBox = 128 * 128;         // one 128-row x 64-col 16-bit box
-  static constexpr int kTile = (D / 64) * kBox;  // Q / K / V tile
+  static constexpr int kBox = 128 * 128;  // one 128-row x 128-byte box (64 16-bit / 128 8-bit columns)
+  static constexpr int kTile = (kFp8 ? D / 128 : D / 64) * kBox;  // Q / K / V tile
   static constexpr int kQ = 0;
   static constexpr int kK = kQ + kTile;
   static constexpr int kV = kK + kStages * kTile;
@@ -105,12 +106,15 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
-template <int D, bool BF16, bool kCausal>
+// kFp8: q, k, v in e4m3 (kind::f8f6f4 MMAs; P cast to e4m3 before P V);
+// BF16 then selects only the type of out
+template <int D, bool BF16, bool kCausal, bool kFp8>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_fwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
-  using L = Layout<D>;
-  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
+  static_assert(!kFp8 || D == 128, "FP8 tiles are one 128-byte box wide");
+  using L = Layout<D, kFp8>;
+  using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;  // out (and 16-bit inputs)
   extern __shared__ unsigned char smem_raw[];
   const uint32_t base = smem_u32(smem_raw);
   unsigned char *sbase = smem_raw;
@@ -223,18 +227,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // is done (S_free).  Each warp runs its loop warp-uniformly (descriptors
     // precomputed and advanced by adding to their address field) and one
     // elected lane issues each MMA and commit.
-    constexpr uint32_t idS = idesc_f16(BF16, 128, 128, false, false);
-    constexpr uint32_t idPV = idesc_f16(BF16, 128, D, false, true);
-    // descriptors: K-major Q / K (a 16-element K step is +32 B, the second
-    // 64-column box +16 KB); MN-major V (a 16-row K step is +2 KB, the two
-    // 64-column halves 16 KB apart)
+    // (format 0 is E4M3 under kind::f8f6f4)
+    constexpr uint32_t idS = idesc_f16(kFp8 ? false : BF16, 128, 128, false, false);
+    constexpr uint32_t idPV = idesc_f16(kFp8 ? false : BF16, 128, D, false, true);
+    // descriptors: K-major Q / K (a K step, 16 16-bit or 32 8-bit elements, is
+    // +32 B; the second 64-column 16-bit box +16 KB); MN-major V (a K step is
+    // 16 rows = +2 KB, or 32 rows = +4 KB for 8-bit; the two 64-column 16-bit
+    // halves 16 KB apart)
+    constexpr int kSSteps = kFp8 ? D / 32 : D / 16;
+    constexpr int kPVSteps = kFp8 ? 4 : 8;
     const uint64_t dQ = sw128_desc(sQ, 16, 1024);
     const uint64_t dK = sw128_desc(sK, 16, 1024);
     const uint64_t dV = sw128_desc(sV, L::kBox, 1024);
     auto kstep = [](int kk) { return uint64_t((kk >> 2) * (L::kBox >> 4) + (kk & 3) * 2); };
-    // 16 kv columns of P = 8 TMEM columns; the first 64 kv columns' P is in
-    // TMEM columns [0, 32), the next 64's in [64, 96) of the S buffer
-    auto pcol = [](int kk) { return uint32_t(64 * (kk >> 2) + 8 * (kk & 3)); };
+    // 16 16-bit (or 32 8-bit) kv columns of P = 8 TMEM columns; the first 64
+    // kv columns' P is in TMEM columns [0, 32) ([0, 16) for 8-bit), the next
+    // 64's in [64, 96) ([64, 80)) of the S buffer
+    auto pcol = [](int kk) {
+      return kFp8 ? uint32_t(64 * (kk >> 1) + 8 * (kk & 1)) : uint32_t(64 * (kk >> 2) + 8 * (kk & 3));
+    };
     const bool is_s = warp == kSMmaWarp;
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
@@ -256,7 +267,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t da = tS0 + uint32_t(b) * 128u;
           const uint64_t ka = dK + uint64_t(st * (L::kTile >> 4));
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) mma_ss_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kSSteps; ++kk) {
+            if constexpr (kFp8) mma_ss_f8_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+            else mma_ss_e(da, dQ + kstep(kk), ka + kstep(kk), idS, kk > 0 ? 1u : 0u);
+          }
           mma_commit_e(bar(kBarSFull + b));
           mma_commit_e(bar(kBarKEmpty + st));
           if (j == n - 1) mma_commit_e(bar(kBarQEmpty));
@@ -273,8 +287,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t pa = tS0 + uint32_t(b) * 128u;
           const uint64_t vd = dV + uint64_t(st * (L::kTile >> 4));
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_ts_e(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (j == 0 && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < kPVSteps; ++kk)
+            if constexpr (kFp8) mma_ts_f8_e(tO, pa + pcol(kk), vd + uint64_t(kk * 256), idPV, (j == 0 && kk == 0) ? 0u : 1u);
+            else mma_ts_e(tO, pa + pcol(kk), vd + uint64_t(kk * 128), idPV, (j == 0 && kk == 0) ? 0u : 1u);
           mma_commit_e(bar(kBarPVDone + int(t & 1u)));
           mma_commit_e(bar(kBarVEmpty + st));
           mma_commit_e(bar(kBarSFree + b));
@@ -344,8 +359,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int st = int(kv_it % kStages);
             if (!(ok = wait_warp(bar(kBarVFull + st), (kv_it / kStages) & 1u, abort, p.status))) break;
             uint4 *vt = reinterpret_cast<uint4 *>(sbase + L::kV + st * L::kTile);
-            const int per_half = (128 - valid_all) * 8;  // 16-byte words per 64-column half
-            for (int w = tid; w < per_half * (D / 64); w += kSoftmaxThreads) {
+            const int per_half = (128 - valid_all) * 8;  // 16-byte words per 128-byte box
+            for (int w = tid; w < per_half * (L::kTile / L::kBox); w += kSoftmaxThreads) {
               const int h = w / per_half, x = w % per_half;
               vt[h * (L::kBox / 16) + valid_all * 8 + x] = make_uint4(0, 0, 0, 0);
             }
@@ -373,7 +388,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               const float e0 = poly ? exp2_poly(a0) : ex2(a0);
               const float e1 = poly ? exp2_poly(a1) : ex2(a1);
               ps[(c >> 1) & 1] += e0 + e1;
-              pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+              if constexpr (kFp8) {
+                // P in e4m3, four to a 32-bit column (the pair before is in
+                // pk[c >> 2]'s low half until this pair completes it)
+                if ((c & 2) == 0) pk[c >> 2] = __float_as_uint(e0), pk[(c >> 2) + kCols / 4] = __float_as_uint(e1);
+                else pk[c >> 2] = pack_e4m3x4(__uint_as_float(pk[c >> 2]), __uint_as_float(pk[(c >> 2) + kCols / 4]), e0, e1);
+              } else {
+                pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+              }
             }
           };
           const bool first = m == -INFINITY;
@@ -438,7 +460,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // P over the first half of this group's own S columns: no other
           // warp reads them any more (the grow path's reads of the other
           // group's S precede its rendezvous)
-          tmem_st_cols<kCols / 2>(tS + uint32_t(kCols * wg), pk);
+          tmem_st_cols<kFp8 ? kCols / 4 : kCols / 2>(tS + uint32_t(kCols * wg), pk);
           l = l * alpha + (ps[0] + ps[1]);
           if (grow && (kCausal || !first) && __any_sync(0xffffffffu, (!kCausal || !first) && alpha != 1.f)) {
             // O may only be rescaled once P_{t-1} V_{t-1} (and so every
@@ -516,16 +538,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool kCausal>
+template <int D, bool BF16, bool kCausal, bool kFp8 = false>
 cudaError_t launch_tc(const Problem &p, const FwdMaps &m, cudaStream_t s) {
   // at least 120 KB so that exactly one CTA (the sole owner of all 512 TMEM
   // columns) is resident per SM
-  const int smem = Layout<D>::kAlloc > 120 * 1024 ? Layout<D>::kAlloc : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16, kCausal>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  const int smem = Layout<D, kFp8>::kAlloc > 120 * 1024 ? Layout<D, kFp8>::kAlloc : 120 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16, kCausal, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.fwd_slots < num_sms() ? p.fwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_fwd_tc<D, BF16, kCausal><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
+  k_fwd_tc<D, BF16, kCausal, kFp8><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
   return cudaGetLastError();
 }
 
@@ -535,8 +557,13 @@ cudaError_t launch_fwd_main(const Problem &p, cudaStream_t s) {
   FwdMaps m;
   cudaError_t e = make_fwd_maps(p, m);
   if (e != cudaSuccess) return e;
-  // the causal mask is a separate instantiation: the unmasked kernel carries
-  // none of its arithmetic
+  // the causal mask and the e4m3 inputs are separate instantiations: the
+  // plain kernel carries neither
+  if (p.dtype == BSA_F8E4M3) {  // D = 128 (checked on the host); out_dtype picks the output type
+    const bool ob = p.out_dtype == BSA_BF16;
+    if (p.causal) return ob ? launch_tc<128, true, true, true>(p, m, s) : launch_tc<128, false, true, true>(p, m, s);
+    return ob ? launch_tc<128, true, false, true>(p, m, s) : launch_tc<128, false, false, true>(p, m, s);
+  }
   if (p.causal) {
     if (p.dtype == BSA_BF16)
       return p.D == 64 ? launch_tc<64, true, true>(p, m, s) : launch_tc<128, true, true>(p, m, s);

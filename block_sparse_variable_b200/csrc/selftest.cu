@@ -4,6 +4,7 @@
 
 #include "bsa_internal.h"
 #include "exp2_poly.cuh"
+#include "fp8.cuh"
 #include "ptx_sm80.cuh"
 #include "tc_device.cuh"
 
@@ -37,6 +38,14 @@ __global__ void k_wait_timeout(uint32_t *flags) {
   if (threadIdx.x == 0 && ok) atomicOr(flags + kStFlags, 0x80000000u);
 }
 
+// groups of four floats -> one word of four e4m3 bytes, as the FP8 forward
+// packs P
+__global__ void k_e4m3_pack(const float *x, uint32_t *y, int64_t nwords) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; i < nwords;
+       i += int64_t(gridDim.x) * blockDim.x)
+    y[i] = pack_e4m3x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
+}
+
 }  // namespace
 }  // namespace bsa
 
@@ -54,5 +63,15 @@ extern "C" bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_
   const int64_t blocks = (n + 255) / 256 < 1024 ? (n + 255) / 256 : 1024;
   bsa::k_exp2_pair<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly,
                                                                                     y_mufu, n);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
+extern "C" bsa_status bsa_selftest_e4m3(const float *x, uint32_t *packed, int64_t n, void *stream) {
+  if (n < 0 || n % 4 != 0) return BSA_ERR_PARAM_INVALID;
+  if (n == 0) return BSA_OK;
+  if (!x || !packed) return BSA_ERR_NULLPTR;
+  const int64_t w = n / 4;
+  const int64_t blocks = (w + 255) / 256 < 1024 ? (w + 255) / 256 : 1024;
+  bsa::k_e4m3_pack<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, packed, w);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }

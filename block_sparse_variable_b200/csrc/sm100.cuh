@@ -181,6 +181,28 @@ __device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint6
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// kind::f8f6f4 (8-bit A and B, fp32 accumulation; a K step is 32 elements):
+// the same two forms, issued by one elected lane
+__device__ __forceinline__ void mma_ss_f8_e(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_f8_e(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_e(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -281,7 +303,9 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo_byte
 
 // Instruction descriptor, kind::f16 with fp32 accumulation: c_format [4,6)
 // = 1 (F32); a/b format [7,10)/[10,13): 0 = F16, 1 = BF16; a/b major bits 15
-// / 16 (1 = MN-major); N >> 3 at [17,23); M >> 4 at [24,29).
+// / 16 (1 = MN-major); N >> 3 at [17,23); M >> 4 at [24,29).  The same
+// fields serve kind::f8f6f4, where format 0 is E4M3 (so idesc_f16(false, ...)
+// describes e4m3 x e4m3 with fp32 accumulation).
 __host__ __device__ constexpr uint32_t idesc_f16(bool bf16, int M, int N, bool a_mn, bool b_mn) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
          ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) | (uint32_t(N >> 3) << 17) |

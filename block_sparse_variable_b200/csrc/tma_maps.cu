@@ -30,18 +30,22 @@ EncodeTiled encoder() {
   return fn;
 }
 
-// 16-bit tiles: 5-D {64 columns, rows, D/64 column halves, heads, batch or
-// page}; one box {64, 128, D/64, 1, 1} lands as D/64 consecutive 128-row x
-// 64-column boxes (16 KB each, 128-byte swizzle), i.e. a whole 128-row tile
-// in one copy.
+// bytes per element of q / k / v
+int64_t esz(const Problem &p) { return p.dtype == BSA_F8E4M3 ? 1 : 2; }
+
+// Tiles of 128-byte rows: 5-D {128-byte column groups (64 16-bit or 128
+// 8-bit columns), rows, D*esz/128 groups, heads, batch or page}; one box
+// {128/esz, 128, D*esz/128, 1, 1} lands as consecutive 128-row x 128-byte
+// boxes (16 KB each, 128-byte swizzle), i.e. a whole 128-row tile in one copy.
 cudaError_t encode(CUtensorMap *m, const Problem &p, const void *base, const cuuint64_t dims[5],
                    const cuuint64_t strides[4]) {
   EncodeTiled fn = encoder();
   if (!fn) return cudaErrorNotSupported;
-  const cuuint32_t box[5] = {64, 128, cuuint32_t(p.D / 64), 1, 1};
+  const cuuint32_t box[5] = {cuuint32_t(128 / esz(p)), 128, cuuint32_t(p.D * esz(p) / 128), 1, 1};
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  const CUtensorMapDataType dt =
-      p.dtype == BSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUtensorMapDataType dt = p.dtype == BSA_F8E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                 : p.dtype == BSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                       : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
   CUresult r = fn(m, dt, 5, const_cast<void *>(base), dims, strides, box, es,
                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -65,30 +69,33 @@ cuuint64_t nz(int64_t x) { return x > 0 ? cuuint64_t(x) : 16; }
 
 cudaError_t kv_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb, int64_t sh,
                    int64_t st) {
-  const cuuint64_t halves = cuuint64_t(p.D / 64);
+  const int64_t e = esz(p);
+  const cuuint64_t inner = cuuint64_t(128 / e), halves = cuuint64_t(p.D * e / 128);
   if (p.kv_layout == BSA_LAYOUT_PA_BBND) {
-    // {64, page rows, halves, kv heads, pages}
-    const cuuint64_t dims[5] = {64, cuuint64_t(p.page_size), halves, cuuint64_t(p.N2), cuuint64_t(p.num_pages)};
-    const cuuint64_t strides[4] = {nz(st * 2), 128, nz(sh * 2), nz(sb * 2)};
+    // {128 B, page rows, groups, kv heads, pages}
+    const cuuint64_t dims[5] = {inner, cuuint64_t(p.page_size), halves, cuuint64_t(p.N2), cuuint64_t(p.num_pages)};
+    const cuuint64_t strides[4] = {nz(st * e), 128, nz(sh * e), nz(sb * e)};
     return encode(m, p, base, dims, strides);
   }
-  // {64, token rows, halves, kv heads, batch}
+  // {128 B, token rows, groups, kv heads, batch}
   const int64_t rows = p.kv_layout == BSA_LAYOUT_TND ? p.Tkv : p.Skv;
   const int64_t nb = p.kv_layout == BSA_LAYOUT_TND ? 1 : p.B;
-  const cuuint64_t dims[5] = {64, cuuint64_t(rows), halves, cuuint64_t(p.N2), cuuint64_t(nb)};
-  const cuuint64_t strides[4] = {nz(st * 2), 128, nz(sh * 2),
-                                 nz(p.kv_layout == BSA_LAYOUT_TND ? rows * st * 2 : sb * 2)};
+  const cuuint64_t dims[5] = {inner, cuuint64_t(rows), halves, cuuint64_t(p.N2), cuuint64_t(nb)};
+  const cuuint64_t strides[4] = {nz(st * e), 128, nz(sh * e),
+                                 nz(p.kv_layout == BSA_LAYOUT_TND ? rows * st * e : sb * e)};
   return encode(m, p, base, dims, strides);
 }
 
 cudaError_t q_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb, int64_t sh,
                   int64_t st) {
-  // {64, token rows, halves, q heads, batch}
+  // {128 B, token rows, groups, q heads, batch}
+  const int64_t e = esz(p);
   const int64_t rows = p.q_layout == BSA_LAYOUT_TND ? p.Tq : p.Sq;
   const int64_t nb = p.q_layout == BSA_LAYOUT_TND ? 1 : p.B;
-  const cuuint64_t dims[5] = {64, cuuint64_t(rows), cuuint64_t(p.D / 64), cuuint64_t(p.N1), cuuint64_t(nb)};
-  const cuuint64_t strides[4] = {nz(st * 2), 128, nz(sh * 2),
-                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * st * 2 : sb * 2)};
+  const cuuint64_t dims[5] = {cuuint64_t(128 / e), cuuint64_t(rows), cuuint64_t(p.D * e / 128), cuuint64_t(p.N1),
+                              cuuint64_t(nb)};
+  const cuuint64_t strides[4] = {nz(st * e), 128, nz(sh * e),
+                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * st * e : sb * e)};
   return encode(m, p, base, dims, strides);
 }
 

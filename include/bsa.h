@@ -54,7 +54,8 @@ enum {
   BSA_F32 = 3,
   BSA_U16 = 4,
   BSA_I32 = 5,
-  BSA_I64 = 6
+  BSA_I64 = 6,
+  BSA_F8E4M3 = 7  /* OCP 8-bit float E4M3 (forward q/k/v only) */
 };
 
 /* A strided view of device memory.  data == NULL (or a NULL descriptor
@@ -120,7 +121,8 @@ typedef enum bsa_status {
 
 /* ------------------------------------------------------------- forward */
 /* Arguments:
- *   q       BNSD [B,N1,Sq,D] or TND [Tq,N1,D], F16 or BF16, D in {64, 128}
+ *   q       BNSD [B,N1,Sq,D] or TND [Tq,N1,D], F16 or BF16, D in {64, 128};
+ *           or F8E4M3 with D = 128 (see below)
  *   k, v    BNSD [B,N2,Skv,D], TND [Tkv,N2,D] or PA_BBND [P,page,N2,D];
  *           same dtype as q; page % 128 == 0
  *   index   U16. BNSD q: [B, Hidx, ceil(Sq/BQ), W]; TND q: [Hidx, R, W] with
@@ -134,9 +136,19 @@ typedef enum bsa_status {
  *                  past seqused_kv[b] are ignored.
  *   block_table    I32 [B, max_pages], required for PA_BBND
  *   out     same shape/dtype as q (written for every q row; rows with no
- *           selected key get 0)
+ *           selected key get 0); F16 or BF16 for F8E4M3 inputs, and then
+ *           its dtype is the output type
  *   lse     F32, BNSD [B,N1,Sq] / TND [Tq,N1]; required when return_lse
  *           (rows with no selected key get -inf)
+ * FP8 inputs (GenericBlockSparseAttention article, quantization table,
+ * quantType 5): q, k, v in E4M3 without scale tensors; the scores are exact
+ * e4m3 products summed in fp32, and P is cast to E4M3 (round to nearest
+ * even, saturating) before the P V product, while the row sums l and lse
+ * come from the unrounded fp32 P.  Each output element then lies within
+ * sum_u (2^-4 P_u + 2^-10) |v_u| / l of the exact result (P_u relative to
+ * the row maximum), plus the output's own rounding.  Strides of FP8
+ * tensors are multiples of 16 elements.  The backward takes 16-bit inputs
+ * only (BSA_ERR_UNSUPPORTED for E4M3).
  */
 bsa_status bsa_fwd_get_workspace(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v,
                                  const bsa_tensor *index, const bsa_tensor *cu_seqlens_q,
@@ -293,6 +305,12 @@ bsa_status bsa_set_main_kernel_events(void *before, void *after);
  * BSA_ERR_NULLPTR for a NULL buffer with n > 0, BSA_ERR_PARAM_INVALID for
  * n < 0, BSA_ERR_CUDA if the launch fails. */
 bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64_t n, void *stream);
+
+/* Diagnostic (the pages have no counterpart).  Packs x[4i .. 4i+3] into
+ * packed[i] as four E4M3 bytes (element 4i in the lowest byte; round to
+ * nearest even, saturating to +-448), with the same routine the FP8 forward
+ * uses for P.  n % 4 == 0; device pointers; asynchronous on `stream`. */
+bsa_status bsa_selftest_e4m3(const float *x, uint32_t *packed, int64_t n, void *stream);
 
 /* Diagnostic (the pages have no counterpart).  Launches one warp that waits
  * on a device barrier nothing ever completes, through the bounded wait every

@@ -35,6 +35,8 @@ def opt_kwargs(d):
 
 def gpu_fwd(p, d=None, out=None, lse=None):
     d = d or device_inputs(p)
+    if out is None and getattr(p, "out_dtype", None) is not None:
+        out = torch.empty(d["q"].shape, dtype=p.out_dtype, device=d["q"].device)
     out, lse, ws = bsa.bsa_fwd(d["q"], d["k"], d["v"], d["index"], params_of(p), out=out, lse=lse,
                                **opt_kwargs(d))
     return out, lse, ws, d

@@ -188,3 +188,33 @@ def test_deterministic_backward_workspace():
     assert bsa.bsa_bwd_get_workspace(p.q, p.k, p.v, p.q, p.dout, lse, p.index, Pd, **kw) \
         == lay_d.total_bytes
     assert _ws(p, params=Pd) == _ws(p)
+
+
+def test_fp8_inputs_forward_only():
+    """e4m3 q/k/v: out must be f16/bf16 (its dtype is the output type), D must
+    be 128, strides 16-byte multiples; the backward refuses them."""
+    p = _prob(D=128, dtype=torch.float8_e4m3fn)
+    P = params_of(p)
+    kw = dict(cu_seqlens_q=p.cu_q, cu_seqlens_kv=p.cu_kv)
+    out_bf = torch.empty(p.q.shape, dtype=torch.bfloat16)
+    out_h = torch.empty(p.q.shape, dtype=torch.float16)
+    lse = torch.empty(p.q.shape[0], p.N1)
+    n = bsa.bsa_fwd_get_workspace(p.q, p.k, p.v, p.index, P, out=out_bf, lse=lse, **kw)
+    assert n > 0
+    assert bsa.bsa_fwd_get_workspace(p.q, p.k, p.v, p.index, P, out=out_h, lse=lse, **kw) == n
+    fp8_out = torch.empty(p.q.shape, dtype=torch.float8_e4m3fn)
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(p.q, p.k, p.v, p.index, P, out=fp8_out, lse=lse,
+                                                   **kw)) == 161002
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(p.q, p.k.to(torch.bfloat16), p.v, p.index, P,
+                                                   out=out_bf, lse=lse, **kw)) == 161002
+    p64 = _prob(D=64, dtype=torch.float8_e4m3fn)
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(
+        p64.q, p64.k, p64.v, p64.index, params_of(p64),
+        out=torch.empty(p64.q.shape, dtype=torch.bfloat16), lse=lse,
+        cu_seqlens_q=p64.cu_q, cu_seqlens_kv=p64.cu_kv)) == 161003
+    wide = torch.zeros(p.q.shape[0], p.q.shape[1], 136, dtype=torch.float8_e4m3fn)[..., :128]
+    assert _code(lambda: bsa.bsa_fwd_get_workspace(wide, p.k, p.v, p.index, P, out=out_bf, lse=lse,
+                                                   **kw)) == 161002       # row stride 136
+    with pytest.raises(bsa.BsaError) as e:
+        bsa.bsa_bwd_get_workspace(p.q, p.k, p.v, out_bf, out_bf, lse, p.index, P, **kw)
+    assert e.value.status == 161003

@@ -374,3 +374,71 @@ def test_configs_full_size_sampled(c):
     assert np.array_equal(H.region(ws_b, lay_b.bwd_items, torch.int32, int(stb[4])), Bld["bwd_items"])
     nnz = int(stb[6])
     assert np.array_equal(H.region(ws_b, lay_b.inv_list, torch.int32, nnz), Bld["inv_list"])
+
+
+# ------------------------------------------------------------- FP8 forward
+# q, k, v in e4m3, P cast to e4m3 before P V (GenericBlockSparseAttention,
+# quantization table, quantType 5); out within the P-cast bound of the exact
+# oracle (tests/harness.py, fp8_out_bound), lse within 1e-3
+FP8 = {
+    "fp8_bnsd_dense": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=128, Sq=640,
+                           pattern=pat_dense),
+    "fp8_bnsd_ragged_kv": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=1, D=128, Sq=300,
+                               lens_kv=[300, 170], Skv=300, pattern=pat_density(0.6, 1)),
+    "fp8_tnd_gqa_fp16_out": dict(layout_q="TND", layout_kv="TND", B=3, N1=4, N2=2, D=128,
+                                 lens_q=[130, 300, 77], lens_kv=[200, 129, 256],
+                                 out_dtype=torch.float16, pattern=pat_random_k),
+    "fp8_paged": dict(layout_q="TND", layout_kv="PA_BBND", B=2, N1=4, N2=2, D=128,
+                      lens_q=[300, 129], lens_kv=[456, 129], page_size=128, extra_pages=2,
+                      pattern=pat_topk(2)),
+    "fp8_big_blocks": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=2, D=128, BQ=256,
+                           BKV=512, lens_q=[700, 300], lens_kv=[900, 300], pattern=pat_random_k),
+    "fp8_causal": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=128,
+                       lens_q=[300, 140], lens_kv=[500, 140], pattern=pat_dense, causal=True),
+    "fp8_empty_rows": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=128,
+                           lens_q=[384, 200], lens_kv=[256, 300], pattern=pat_random_k,
+                           row_hook=_hook_empty),
+}
+
+
+def _fp8_problem(name):
+    return make_problem(seed_base=zlib.crc32(name.encode()) % 9973, name=name,
+                        dtype=torch.float8_e4m3fn, **FP8[name])
+
+
+def _check_fp8(p):
+    out_ref, lse_ref, fl = oracle.Oracle(p).fwd()
+    d = H.device_inputs(p)
+    out, lse, ws, _ = H.gpu_fwd(p, d)
+    torch.cuda.synchronize()
+    assert out.dtype == p.odtype
+    H.check_fp8_out(out, out_ref, H.fp8_out_bound(p), p.odtype)
+    H.check_lse(lse, lse_ref)
+    assert bsa.bsa_read_status(ws) == (fl | oracle.Oracle(p).scan_flags())
+
+
+@pytest.mark.parametrize("name", sorted(FP8))
+def test_fp8_forward(name):
+    _check_fp8(_fp8_problem(name))
+
+
+def test_fp8_forward_nan_in_unused_kv_rows():
+    p = _poison_unused_kv(_fp8_problem("fp8_paged"))
+    assert torch.isnan(p.k.float()).any()
+    _check_fp8(p)
+
+
+def test_fp8_pack_is_round_to_nearest_even():
+    """The kernel's P packing against torch's fp32 -> e4m3 conversion, byte
+    order included; out-of-range values saturate to +-448."""
+    g = torch.Generator().manual_seed(5)
+    x = torch.cat([torch.randn(4096, generator=g) * 4,
+                   torch.rand(4096, generator=g) * 2.0 ** -6,         # subnormal range
+                   torch.tensor([0.0, -0.0, 448.0, -448.0, 2.0 ** -10, 3 * 2.0 ** -10,
+                                 1.0625, 1.1875, 240.0, 2.0 ** -9])])
+    x = x[: (x.numel() // 4) * 4]
+    got = bsa.bsa_selftest_e4m3(x.cuda()).cpu()
+    ref = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    assert torch.equal(got, ref)
+    sat = bsa.bsa_selftest_e4m3(torch.tensor([1000.0, -1000.0, 449.0, 0.5]).cuda()).cpu()
+    assert sat.tolist() == [0x7E, 0xFE, 0x7E, 0x30]
