@@ -149,21 +149,21 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- oracle leg
-def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False):
+def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = False):
     """A bounded slice of the workload for the CPU oracle: batch 0, head 0,
     the first q_rows query rows against the full key range (causal: the
     last q_rows rows, which keeps every row's place relative to the end of
     the kv sequence)."""
     import workloads
     from workloads.gen import make_problem, pat_dense
-    p = workloads.make_config(cfg, causal=causal)
+    p = workloads.make_config(cfg, causal=causal, fp8=fp8)
     if p.layout_q != "BNSD":
         raise SystemExit("CPU baseline slice is defined for the BNSD workloads")
     S = p.q.shape[2]
     q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
     sub = make_problem(B=1, N1=1, N2=1, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
                        BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale,
-                       causal=causal)
+                       causal=causal, out_dtype=p.out_dtype)
     rows = slice(S - q_rows, S) if causal else slice(0, q_rows)
     blocks = slice(rows.start // p.BQ, rows.stop // p.BQ)
     sub.q = p.q[:1, :1, rows].contiguous()
@@ -420,6 +420,108 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_fp8(args):
+    """C3 with e4m3 q, k, v (bf16 out): the forward alone (the backward takes
+    16-bit inputs), timed like run_ours; the roofline peak is the measured
+    bf16 burst x 2 (the nominal fp8 / bf16 tensor ratio, 4.5 / 2.25 PFLOP/s)."""
+    import block_sparse_variable_b200 as bsa
+    import workloads
+    from tests.harness import params_of
+
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    p = workloads.make_config(3, fp8=True)
+    pairs = _pairs(p)
+    P = params_of(p)
+    q, k, v, index = (getattr(p, n).to(dev) for n in ("q", "k", "v", "index"))
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
+    wsf = torch.empty(bsa.bsa_fwd_get_workspace(q, k, v, index, P, out=out, lse=lse),
+                      dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        bsa.bsa_fwd(q, k, v, index, P, out=out, lse=lse, workspace=wsf, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    flags = bsa.bsa_read_status(wsf)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for e in (e for row in kev for e in row):
+        e.record(stream)
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with ClockSampler(0) as clk:
+        start.record(stream)
+        for s_ in range(args.steps):
+            ev[s_][0].record(stream)
+            bsa.bsa_set_main_kernel_events(kev[s_][0], kev[s_][1])
+            step()
+            ev[s_][1].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize()
+    ms = start.elapsed_time(stop) / args.steps
+    kms = statistics.mean(e[0].elapsed_time(e[1]) for e in kev)
+    # end to end: q, k, v, index in from pinned host memory, out and lse back
+    hq, hk, hv, hidx = (t.cpu().pin_memory() for t in (q, k, v, index))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hidx))
+    d2h = sum(t.numel() * t.element_size() for t in (h_out, h_lse))
+
+    def e2e_step():
+        for d_, h_ in ((q, hq), (k, hk), (v, hv), (index, hidx)):
+            d_.copy_(h_, non_blocking=True)
+        step()
+        for h_, d_ in ((h_out, out), (h_lse, lse)):
+            h_.copy_(d_, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(2, min(args.steps, 5))
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    peaks, which = _peaks()
+    flops = 4 * p.D * pairs
+    peak = 2 * peaks["bf16_tflops"]
+    ktf = flops / (kms * 1e-3) / 1e12
+    line = {
+        "metric": "effective TFLOP/s (selected blocks only), FP8 forward", "value": round(flops / (ms * 1e-3) / 1e12, 3),
+        "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3", "data": "synthetic",
+        "config": {"workload": DESCR[3] + ", q/k/v e4m3 (bf16 out), forward only",
+                   "kept_pairs_per_replica": pairs, "parallelism": "replicas x1 (no exchange)",
+                   "l2": "inputs larger than L2 (q/k/v %d MiB each)" % (q.numel() >> 20)},
+        "kernel_ms": {"k_fwd_tc": round(kms, 4)}, "kernel_tflops": {"k_fwd_tc": round(ktf, 2)},
+        "roofline": {"bound": "tensor", "kernel": "k_fwd_tc", "units": "4*D*kept_pairs FLOPs per launch",
+                     "achieved": round(ktf, 2), "peak": peak, "unit": "TFLOP/s",
+                     "frac": round(ktf / peak, 4),
+                     "peak_source": f"{which} bf16 burst x 2 (nominal fp8/bf16 ratio)", "traffic": None},
+        "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
+        "gpu_launches": 5 * args.steps, "status_flags": flags, "clocks": clk.summary(),
+    }
+    if not args.no_cpu_baseline:
+        sub = _oracle_subproblem(3, 8192, fp8=True)
+        import oracle
+        t = time.perf_counter()
+        oracle.Oracle(sub).fwd()
+        t = time.perf_counter() - t
+        line["cpu_baseline"] = {"value": 4 * sub.D * _pairs(sub) / t / 1e12, "unit": "TFLOP/s",
+                                "cores": _omp_threads(), "kind": "oracle",
+                                "sample": f"fp64 oracle forward on batch 0, head 0, first "
+                                          f"{sub.q.shape[2]} query rows x {sub.k.shape[2]} keys ({t:.1f} s)"}
+    print(json.dumps(line), flush=True)
+
+
 def _traffic_from_profiles(cfg, which):
     """DRAM bytes per launch of the dominant kernel from a committed ncu summary."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
@@ -445,11 +547,15 @@ def main():
                     help="C3 with the causal mask and its lower-triangular block index")
     ap.add_argument("--deterministic", action="store_true",
                     help="the deterministic backward (bitwise reproducible dq)")
+    ap.add_argument("--fp8", action="store_true",
+                    help="C3 with e4m3 q/k/v: the FP8 forward alone (one GPU)")
     args = ap.parse_args()
     if args.causal and args.config != 3:
         ap.error("--causal applies to C3")
     if args.impl == "reference":
         run_reference(args)
+    elif args.fp8:
+        run_fp8(args)
     else:
         run_ours(args)
 

@@ -264,12 +264,16 @@ def _lens(seed, B, lo, hi):
     return [int(x) for x in rng.integers(lo, hi + 1, size=B)]
 
 
-def make_config(c: int, batch: int | None = None, causal: bool = False) -> Problem:
+def make_config(c: int, batch: int | None = None, causal: bool = False, fp8: bool = False) -> Problem:
     """C1..C5: the five workload shapes (see the module docstring for seeds).
 
     `batch` overrides the batch of the BNSD shapes C3 and C4 (smaller cases
     of the same kernels for profiler captures).  `causal` turns C3 into its
-    causal variant: the causal mask with the lower-triangular block index."""
+    causal variant: the causal mask with the lower-triangular block index;
+    `fp8` gives C3 e4m3 q, k, v (bf16 out), the same N(0,1) draws rounded to
+    e4m3."""
+    if fp8 and c != 3:
+        raise ValueError("the FP8 variant is defined for C3 only")
     if batch is not None and c not in (3, 4):
         raise ValueError("batch override applies to C3 and C4 only")
     if causal and c != 3:
@@ -288,7 +292,8 @@ def make_config(c: int, batch: int | None = None, causal: bool = False) -> Probl
         return make_problem(name="C3-causal" if causal else "C3", layout_q="BNSD", layout_kv="BNSD",
                             B=batch or 2, N1=32, N2=32, D=128, Sq=8192, BQ=128, BKV=512, W=16,
                             pattern=pat_causal_blocks(128, 512) if causal else pat_dense,
-                            seed_base=s, causal=causal)
+                            seed_base=s, causal=causal,
+                            dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
     if c == 4:
         return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=batch or 1, N1=24, N2=24, D=128,
                             Sq=32768, BQ=128, BKV=128, W=256, pattern=pat_sink_diag_random(14),
