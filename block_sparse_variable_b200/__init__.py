@@ -1,7 +1,7 @@
 """Block-sparse variable-length FlashAttention for B200 (sm_100a).
 
 Thin ctypes binding over the C ABI in ``include/bsa.h`` (``libbsa.so``,
-built in-tree by ``block_sparse_variable_b200.build``).  The functions keep
+built in-tree by ``block_sparse_variable_b200/build.py``).  The functions keep
 the C names; they only marshal torch tensors into ``bsa_tensor``
 descriptors, allocate outputs / workspace with torch when the caller does
 not pass them, and raise ``BsaError`` on a non-OK status.  Every step of
@@ -65,7 +65,7 @@ class bsa_ws_layout(ctypes.Structure):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with "
-                          f"`python -m block_sparse_variable_b200.build` (nvcc, sm_100a)")
+                          f"`python block_sparse_variable_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     T = ctypes.POINTER(bsa_tensor)
     Pp = ctypes.POINTER(bsa_params)
