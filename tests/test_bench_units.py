@@ -1,0 +1,48 @@
+"""The benchmark's algorithmic unit: kept (q head, valid q token, visible kv
+token) pairs.  bench._pairs counts them from the index arithmetically; here
+the count is checked against the dense token mask (torch_reference) on small
+problems of every layout, with and without the causal mask, and the causal
+C3 closed form S(S+1)/2 per head."""
+import sys
+import os
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from tests import torch_reference as TR  # noqa: E402
+from workloads.gen import (make_problem, pat_causal, pat_causal_blocks, pat_dense,  # noqa: E402
+                           pat_fraction_diag, pat_random_k, pat_topk)
+
+CASES = {
+    "bnsd": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=2, N2=1, D=16, Sq=300,
+                 lens_kv=[300, 170], Skv=300, pattern=pat_random_k),
+    "bnsd_blocks": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=2, N2=2, D=16, Sq=700, BQ=256,
+                        BKV=512, pattern=pat_dense),
+    "tnd_gqa_shared": dict(layout_q="TND", layout_kv="TND", B=3, N1=4, N2=2, Hidx=2, D=16,
+                           lens_q=[130, 300, 77], lens_kv=[200, 129, 256],
+                           pattern=pat_fraction_diag(0.5)),
+    "paged": dict(layout_q="TND", layout_kv="PA_BBND", B=2, N1=2, N2=1, D=16,
+                  lens_q=[300, 129], lens_kv=[456, 129], page_size=128, pattern=pat_topk(2)),
+}
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_pairs_count_the_dense_mask(name, causal):
+    p = make_problem(seed_base=11, causal=causal, **CASES[name])
+    dense = sum(int(TR.token_mask(p, b).sum()) for b in range(p.B))
+    assert bench._pairs(p) == dense
+
+
+def test_causal_square_closed_form():
+    S = 1024
+    p = make_problem(layout_q="BNSD", layout_kv="BNSD", B=1, N1=3, N2=3, D=16, Sq=S, BQ=128, BKV=512,
+                     pattern=pat_causal_blocks(128, 512), causal=True, seed_base=3)
+    assert bench._pairs(p) == 3 * S * (S + 1) // 2
+    q = make_problem(layout_q="BNSD", layout_kv="BNSD", B=1, N1=1, N2=1, D=16, Sq=S, BQ=128, BKV=128,
+                     pattern=pat_causal, causal=True, seed_base=3)
+    assert bench._pairs(q) == S * (S + 1) // 2
