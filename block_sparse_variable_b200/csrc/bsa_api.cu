@@ -420,7 +420,7 @@ const char *bsa_status_string(bsa_status s) {
     case BSA_OK: return "BSA_OK";
     case BSA_ERR_NULLPTR: return "BSA_ERR_NULLPTR: a required pointer is NULL";
     case BSA_ERR_PARAM_INVALID: return "BSA_ERR_PARAM_INVALID: shapes, strides, dtypes or attributes disagree";
-    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED: outside what this build supports";
+    case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED: outside what this library supports";
     case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE: workspace NULL, misaligned or too small";
     case BSA_ERR_CUDA: return "BSA_ERR_CUDA: a CUDA launch or call failed";
     case BSA_ERR_INNER: return "BSA_ERR_INNER: internal inconsistency";

@@ -105,7 +105,7 @@ typedef enum bsa_status {
   BSA_OK = 0,
   BSA_ERR_NULLPTR = 161001,       /* a required pointer or descriptor is NULL */
   BSA_ERR_PARAM_INVALID = 161002, /* shapes / strides / dtypes / attributes disagree */
-  BSA_ERR_UNSUPPORTED = 161003,   /* valid request outside what this build supports */
+  BSA_ERR_UNSUPPORTED = 161003,   /* valid request outside what this library supports */
   BSA_ERR_WORKSPACE = 161004,     /* workspace NULL, misaligned or too small */
   BSA_ERR_CUDA = 561000,          /* a kernel launch or CUDA call failed */
   BSA_ERR_INNER = 561103          /* internal inconsistency */
