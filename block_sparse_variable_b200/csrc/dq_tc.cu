@@ -35,6 +35,7 @@
 #include <type_traits>
 
 #include "addr.cuh"
+#include "coalesce.cuh"
 #include "bsa_internal.h"
 #include "fwd_walk.cuh"
 #include "ptx_sm80.cuh"
@@ -369,35 +370,35 @@ __global__ void __launch_bounds__(kDThreads, 1)
         mbar_arrive(bar(kDBarDSFull + b));
       }
       if (!ok) break;
-      // ---- epilogue: dq = dtype(scale * dQ); group w writes D/2 columns
-      T *qrow = static_cast<T *>(p.dq) + q_row(p.dq_sb, p.dq_sh, p.dq_st, v.bi, v.b, v.h1, t);
+      // ---- epilogue: dq = dtype(scale * dQ); group w writes D/2 columns,
+      // stored through an in-warp transpose so that each store writes whole rows
+      constexpr int kC = D / 16;  // 16-byte chunks of a thread's D/2 columns
+      const int wrow = 32 * (warp & 3);  // this warp's first row of the tile
+      uint4 qch[kC];
       if (n > 0) {
         if (!(ok = wait_warp(bar(kDBarDQDone), dq_it & 1u, abort, p.status))) break;
         ++dq_it;
         tc_fence_after();
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
-          const uint32_t col = uint32_t((D / 2) * wg + 32 * h);
           uint32_t x[32];
-          tmem_ld32(tDQ + lane_off + col, x);
+          tmem_ld32(tDQ + lane_off + uint32_t((D / 2) * wg + 32 * h), x);
           tmem_wait_ld();
-          if (live) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 8) {
-              uint4 w;
-              w.x = MmaOp<T>::pack(__uint_as_float(x[c]) * p.scale, __uint_as_float(x[c + 1]) * p.scale);
-              w.y = MmaOp<T>::pack(__uint_as_float(x[c + 2]) * p.scale, __uint_as_float(x[c + 3]) * p.scale);
-              w.z = MmaOp<T>::pack(__uint_as_float(x[c + 4]) * p.scale, __uint_as_float(x[c + 5]) * p.scale);
-              w.w = MmaOp<T>::pack(__uint_as_float(x[c + 6]) * p.scale, __uint_as_float(x[c + 7]) * p.scale);
-              *reinterpret_cast<uint4 *>(qrow + col + c) = w;
-            }
+          for (int c = 0; c < 4; ++c) {
+            qch[4 * h + c].x = MmaOp<T>::pack(__uint_as_float(x[8 * c]) * p.scale, __uint_as_float(x[8 * c + 1]) * p.scale);
+            qch[4 * h + c].y = MmaOp<T>::pack(__uint_as_float(x[8 * c + 2]) * p.scale, __uint_as_float(x[8 * c + 3]) * p.scale);
+            qch[4 * h + c].z = MmaOp<T>::pack(__uint_as_float(x[8 * c + 4]) * p.scale, __uint_as_float(x[8 * c + 5]) * p.scale);
+            qch[4 * h + c].w = MmaOp<T>::pack(__uint_as_float(x[8 * c + 6]) * p.scale, __uint_as_float(x[8 * c + 7]) * p.scale);
           }
         }
-      } else if (live) {
+      } else {
 #pragma unroll
-        for (int c = 0; c < D / 16; ++c)
-          reinterpret_cast<uint4 *>(qrow + (D / 2) * wg)[c] = make_uint4(0, 0, 0, 0);
+        for (int c = 0; c < kC; ++c) qch[c] = make_uint4(0, 0, 0, 0);
       }
+      transpose_chunks<kC>(qch, lane);
+      T *qrow0 = static_cast<T *>(p.dq) + q_row(p.dq_sb, p.dq_sh, p.dq_st, v.bi, v.b, v.h1, v.t0 + wrow) + (D / 2) * wg;
+      store_rows<kC>(qrow0, p.dq_st, v.rows - wrow, qch, lane);
       // dQ is free for the next item once every softmax thread has arrived
       // on that item's first dS_full (the dQ issuer waits for it)
       tc_fence_before();
