@@ -38,7 +38,6 @@
 #include <type_traits>
 
 #include "addr.cuh"
-#include "coalesce.cuh"
 #include "bsa_internal.h"
 #include "ptx_sm80.cuh"
 #include "sm100.cuh"
@@ -530,38 +529,43 @@ __global__ void __launch_bounds__(kBThreads, 1)
       // ---- epilogue: dK * scale and dV, group w writes columns [w*D/2, (w+1)*D/2)
       if (!(ok = wait_warp(bar(kBarAcc), item_n & 1u, abort, p.status))) break;
       tc_fence_after();
-      {
-        // dK * scale and dV (zeros for an item without steps), each stored
-        // through an in-warp transpose so that each store writes whole rows
-        constexpr int kC = D / 16;  // 16-byte chunks of a thread's D/2 columns
-        const int wrow = 32 * (warp & 3);  // this warp's first kv row of the slice
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t tacc = which == 0 ? tdK : tdV;
-          const float sc = which == 0 ? p.scale : 1.f;
-          uint4 q[kC];
-          if (nsteps > 0) {
+      if (r < v.wb) {
+        T *dkr = static_cast<T *>(p.dk) + kv_row(p, p.dk_sb, p.dk_sh, p.dk_st, v.bi, v.b, v.h2, v.u0 + r, v.pg);
+        T *dvr = static_cast<T *>(p.dv) + kv_row(p, p.dv_sb, p.dv_sh, p.dv_st, v.bi, v.b, v.h2, v.u0 + r, v.pg);
+        if (nsteps == 0) {
 #pragma unroll
-            for (int h = 0; h < D / 64; ++h) {
-              uint32_t x[32];
-              tmem_ld32(tacc + lane_off + uint32_t((D / 2) * wg + 32 * h), x);
-              tmem_wait_ld();
-#pragma unroll
-              for (int c = 0; c < 4; ++c) {
-                q[4 * h + c].x = MmaOp<T>::pack(__uint_as_float(x[8 * c]) * sc, __uint_as_float(x[8 * c + 1]) * sc);
-                q[4 * h + c].y = MmaOp<T>::pack(__uint_as_float(x[8 * c + 2]) * sc, __uint_as_float(x[8 * c + 3]) * sc);
-                q[4 * h + c].z = MmaOp<T>::pack(__uint_as_float(x[8 * c + 4]) * sc, __uint_as_float(x[8 * c + 5]) * sc);
-                q[4 * h + c].w = MmaOp<T>::pack(__uint_as_float(x[8 * c + 6]) * sc, __uint_as_float(x[8 * c + 7]) * sc);
-              }
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < kC; ++c) q[c] = make_uint4(0, 0, 0, 0);
+          for (int c = 0; c < D / 16; ++c) {
+            reinterpret_cast<uint4 *>(dkr + (D / 2) * wg)[c] = make_uint4(0, 0, 0, 0);
+            reinterpret_cast<uint4 *>(dvr + (D / 2) * wg)[c] = make_uint4(0, 0, 0, 0);
           }
-          transpose_chunks<kC>(q, lane);
-          T *row0 = which == 0
-                        ? static_cast<T *>(p.dk) + kv_row(p, p.dk_sb, p.dk_sh, p.dk_st, v.bi, v.b, v.h2, v.u0 + wrow, v.pg)
-                        : static_cast<T *>(p.dv) + kv_row(p, p.dv_sb, p.dv_sh, p.dv_st, v.bi, v.b, v.h2, v.u0 + wrow, v.pg);
-          store_rows<kC>(row0 + (D / 2) * wg, which == 0 ? p.dk_st : p.dv_st, v.wb - wrow, q, lane);
+        }
+      }
+      if (nsteps > 0) {
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h) {
+          const uint32_t col = uint32_t((D / 2) * wg + 32 * h);
+          uint32_t xk[32], xv[32];
+          tmem_ld32(tdK + lane_off + col, xk);
+          tmem_ld32(tdV + lane_off + col, xv);
+          tmem_wait_ld();
+          if (r < v.wb) {
+            T *dkr = static_cast<T *>(p.dk) + kv_row(p, p.dk_sb, p.dk_sh, p.dk_st, v.bi, v.b, v.h2, v.u0 + r, v.pg) + col;
+            T *dvr = static_cast<T *>(p.dv) + kv_row(p, p.dv_sb, p.dv_sh, p.dv_st, v.bi, v.b, v.h2, v.u0 + r, v.pg) + col;
+#pragma unroll
+            for (int c = 0; c < 32; c += 8) {
+              uint4 wk, wv;
+              wk.x = MmaOp<T>::pack(__uint_as_float(xk[c]) * p.scale, __uint_as_float(xk[c + 1]) * p.scale);
+              wk.y = MmaOp<T>::pack(__uint_as_float(xk[c + 2]) * p.scale, __uint_as_float(xk[c + 3]) * p.scale);
+              wk.z = MmaOp<T>::pack(__uint_as_float(xk[c + 4]) * p.scale, __uint_as_float(xk[c + 5]) * p.scale);
+              wk.w = MmaOp<T>::pack(__uint_as_float(xk[c + 6]) * p.scale, __uint_as_float(xk[c + 7]) * p.scale);
+              wv.x = MmaOp<T>::pack(__uint_as_float(xv[c]), __uint_as_float(xv[c + 1]));
+              wv.y = MmaOp<T>::pack(__uint_as_float(xv[c + 2]), __uint_as_float(xv[c + 3]));
+              wv.z = MmaOp<T>::pack(__uint_as_float(xv[c + 4]), __uint_as_float(xv[c + 5]));
+              wv.w = MmaOp<T>::pack(__uint_as_float(xv[c + 6]), __uint_as_float(xv[c + 7]));
+              *reinterpret_cast<uint4 *>(dkr + c) = wk;
+              *reinterpret_cast<uint4 *>(dvr + c) = wv;
+            }
+          }
         }
       }
       tc_fence_before();
