@@ -218,3 +218,23 @@ def test_fp8_inputs_forward_only():
     with pytest.raises(bsa.BsaError) as e:
         bsa.bsa_bwd_get_workspace(p.q, p.k, p.v, out_bf, out_bf, lse, p.index, P, **kw)
     assert e.value.status == 161003
+
+
+def test_plain_c_caller():
+    """A C program built against include/bsa.h alone links libbsa.so and
+    sizes workspaces / gets the host refusals (tests/c_abi_check.c)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    pkg = os.path.dirname(bsa.LIB_PATH)
+    out_dir = os.path.join(pkg, "_build")
+    os.makedirs(out_dir, exist_ok=True)
+    exe = os.path.join(out_dir, "c_abi_check")
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           os.path.join(ROOT, "tests", "c_abi_check.c"), "-o", exe,
+                           f"-L{pkg}", "-l:libbsa.so", f"-Wl,-rpath,{pkg}"])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "ok"
