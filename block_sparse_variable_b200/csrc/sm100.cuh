@@ -1,5 +1,5 @@
 // sm100.cuh -- Blackwell (sm_100a) building blocks written as inline PTX:
-// mbarriers with bounded waits, TMA tile loads (no multicast), TMEM
+// mbarriers with bounded waits, TMA tile loads (each CTA loads its own tiles), TMEM
 // allocation, tcgen05.mma (SS and TS forms), tcgen05.commit, TMEM
 // loads/stores, and the shared-memory matrix / instruction descriptors.
 #pragma once
