@@ -238,3 +238,21 @@ def test_plain_c_caller():
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "ok"
+
+
+def test_binding_refuses_to_import_without_the_library():
+    """No fallback: a copy of the binding with no libbsa.so beside it raises
+    ImportError at import (run in a child process)."""
+    import shutil
+    import subprocess
+    import sys
+    pkg = os.path.dirname(bsa.LIB_PATH)
+    root = os.path.join(pkg, "_build", "nolib")
+    shutil.rmtree(root, ignore_errors=True)
+    os.makedirs(os.path.join(root, "block_sparse_variable_b200"))
+    shutil.copy(os.path.join(pkg, "__init__.py"), os.path.join(root, "block_sparse_variable_b200"))
+    r = subprocess.run([sys.executable, "-c", "import block_sparse_variable_b200"], cwd=root,
+                       capture_output=True, text=True, timeout=300,
+                       env=dict(os.environ, PYTHONPATH=root))
+    assert r.returncode != 0
+    assert "ImportError" in r.stderr and "libbsa.so is missing" in r.stderr
