@@ -46,3 +46,17 @@ def test_causal_square_closed_form():
     q = make_problem(layout_q="BNSD", layout_kv="BNSD", B=1, N1=1, N2=1, D=16, Sq=S, BQ=128, BKV=128,
                      pattern=pat_causal, causal=True, seed_base=3)
     assert bench._pairs(q) == S * (S + 1) // 2
+
+
+def test_causal_blocks_pattern_is_exactly_the_reachable_blocks():
+    """C3's causal variant keeps, for query block i, exactly the kv blocks
+    that hold at least one token a row of block i may see."""
+    S, BQ, BKV = 2048, 128, 512
+    p = make_problem(layout_q="BNSD", layout_kv="BNSD", B=1, N1=1, N2=1, D=16, Sq=S, BQ=BQ, BKV=BKV,
+                     pattern=pat_causal_blocks(BQ, BKV), causal=True, seed_base=5)
+    idx = p.index.view(torch.int16).numpy().view("uint16")[0, 0]
+    for i in range(S // BQ):
+        row = sorted(int(e) for e in idx[i] if e != 0xFFFF)
+        last_visible = i * BQ + BQ - 1          # the block's last row sees up to its own token
+        want = list(range(last_visible // BKV + 1))
+        assert row == want, (i, row, want)
