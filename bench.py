@@ -215,21 +215,43 @@ def _omp_threads():
 
 
 def run_reference(args):
+    """The oracle on the host cores, on the same workload, metric and unit as
+    the GPU arm (--causal, --deterministic and --fp8 select the same variant;
+    the deterministic mode changes nothing the oracle computes; --fp8 times
+    the forward alone, as the GPU arm does)."""
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    sub, pairs = _oracle_rate(args.config, 2.0, args.causal)
+    fp8 = getattr(args, "fp8", False)
+    if fp8:
+        sub = _oracle_subproblem(3, 1024, fp8=True)
+        pairs = _pairs(sub)
+
+        def one():
+            import oracle
+            t = time.perf_counter()
+            oracle.Oracle(sub).fwd()
+            return time.perf_counter() - t
+        metric, per_pair = "effective TFLOP/s (selected blocks only), FP8 forward", 4
+        workload = DESCR[3] + ", q/k/v e4m3 (bf16 out), forward only"
+    else:
+        sub, pairs = _oracle_rate(args.config, 2.0, args.causal)
+
+        def one():
+            return _oracle_step(sub)
+        metric, per_pair = METRIC, 14
+        workload = _descr(args.config, args.causal, getattr(args, "deterministic", False))
     for _ in range(args.warmup):
-        _oracle_step(sub)
-    ts = [_oracle_step(sub) for _ in range(args.steps)]
+        one()
+    ts = [one() for _ in range(args.steps)]
     total = sum(ts)
-    flops = 14 * sub.D * pairs
+    flops = per_pair * sub.D * pairs
     val = flops * args.steps / total / 1e12
-    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s",
+    line = {"impl": "reference", "metric": metric, "value": val, "unit": "TFLOP/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": _descr(args.config, args.causal), "sample": "see cpu_baseline"},
+            "config": {"workload": workload, "sample": "see cpu_baseline"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _omp_threads(),
                              "kind": "oracle",
                              "sample": f"batch 0, head 0, {'last' if args.causal else 'first'} "
