@@ -450,6 +450,8 @@ def run_fp8(args):
     import workloads
     from tests.harness import params_of
 
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        raise SystemExit("--fp8 is a one-GPU line; run it without torchrun")
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     p = workloads.make_config(3, fp8=True)
