@@ -63,6 +63,7 @@ def _load():
         _lib.oracle_bwd_dq_rows.argtypes = [P, vp, vp, vp, vp, i64, vp, vp]
         _lib.oracle_bwd_dkv_rows.argtypes = [P, vp, vp, vp, vp, i64, vp, vp, vp]
         _lib.oracle_scan_flags.argtypes = [P, vp]
+        _lib.oracle_batch_lengths.argtypes = [P, vp, vp, vp, vp]
     return _lib
 
 
@@ -109,18 +110,31 @@ class Oracle:
         self._s = s
         self.lib = _load()
 
+    # ---------------------------------------------------------- lengths
+    def batch_lengths(self):
+        """Per batch (query rows, used kv tokens, stored kv rows) and the flag
+        bits the lengths raise; a length that contradicts its storage counts
+        as 0 (bsa_oracle.c, oracle_batch_lengths)."""
+        B = self.prob.B
+        ql, kl, ks = (np.zeros(B, np.int64) for _ in range(3))
+        fl = ctypes.c_uint32(0)
+        self.lib.oracle_batch_lengths(ctypes.byref(self._s), ql.ctypes.data, kl.ctypes.data,
+                                      ks.ctypes.data, ctypes.addressof(fl))
+        return [int(x) for x in ql], [int(x) for x in kl], [int(x) for x in ks], fl.value
+
     # ------------------------------------------------------------- rows
     def q_rows_all(self) -> np.ndarray:
-        """All (b, h1, t) query rows in storage order of the q tensor's rows."""
+        """All (b, h1, t) query rows of every batch (t below the batch's query
+        length), in storage order of the q tensor's rows."""
         p = self.prob
         rows = []
         if p.layout_q == "BNSD":
             S = p.q.shape[2]
             b, h, t = np.meshgrid(np.arange(p.B), np.arange(p.N1), np.arange(S), indexing="ij")
             return np.stack([b.ravel(), h.ravel(), t.ravel()], 1).astype(np.int64)
-        cu = p.cu_q.tolist()
+        qlen = self.batch_lengths()[0]
         for b in range(p.B):
-            L = cu[b + 1] - cu[b]
+            L = qlen[b]
             t, h = np.meshgrid(np.arange(L), np.arange(p.N1), indexing="ij")
             rows.append(np.stack([np.full(t.size, b), h.ravel(), t.ravel()], 1))
         return np.concatenate(rows).astype(np.int64) if rows else np.zeros((0, 3), np.int64)
@@ -201,23 +215,24 @@ class Oracle:
         return dk, dv, fl.value
 
     def kv_rows_all(self) -> np.ndarray:
-        """All (b, h2, u) kv rows with u < the batch's used kv length."""
+        """All (b, h2, u) kv rows with u < the batch's used kv length (paged:
+        whose block-table entry names a page; the tokens of a bad entry have
+        no storage row)."""
         p = self.prob
         lens = self.kv_lens()
         rows = []
         for b in range(p.B):
-            u, h = np.meshgrid(np.arange(lens[b]), np.arange(p.N2), indexing="ij")
+            us = np.arange(lens[b])
+            if p.layout_kv == "PA_BBND":
+                pages = p.block_table[b].numpy().astype(np.int64)[us // p.k.shape[1]]
+                us = us[(pages >= 0) & (pages < p.k.shape[0])]
+            u, h = np.meshgrid(us, np.arange(p.N2), indexing="ij")
             rows.append(np.stack([np.full(u.size, b), h.ravel(), u.ravel()], 1))
         return np.concatenate(rows).astype(np.int64) if rows else np.zeros((0, 3), np.int64)
 
     def kv_lens(self):
-        p = self.prob
-        if p.seqused_kv is not None:
-            return [int(x) for x in p.seqused_kv]
-        if p.layout_kv == "TND":
-            cu = p.cu_kv.tolist()
-            return [cu[b + 1] - cu[b] for b in range(p.B)]
-        return [p.k.shape[2]] * p.B
+        """Used kv tokens per batch (0 where a length contradicts its storage)."""
+        return self.batch_lengths()[1]
 
     def kv_index(self, kvrows: np.ndarray):
         """Advanced-index tuple addressing kv rows (b, h2, u) in the k/v tensor."""

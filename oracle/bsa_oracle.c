@@ -328,6 +328,28 @@ int oracle_bwd_dkv_rows(const oracle_problem *P, const double *out, const double
   return 0;
 }
 
+/* ========================================================= batch lengths */
+/* Per batch: query rows, used kv tokens and stored kv rows as the
+ * definition reads them (GenericBlockSparseAttention, "dual length"
+ * semantics: seqused_kv may not exceed the stored length; a contradictory
+ * length counts as 0 and raises ORACLE_BAD_SEQLEN).  The stored rows are
+ * those of the batch's own kv storage: BNSD Skv, TND the cu_seqlens_kv
+ * difference, PA_BBND the pages that cover the used length. */
+int oracle_batch_lengths(const oracle_problem *P, int64_t *qlen, int64_t *kvlen,
+                         int64_t *kvstored, uint32_t *flags) {
+  uint32_t fl = 0;
+  for (int64_t b = 0; b < P->B; ++b) {
+    qlen[b] = q_len(P, b, &fl);
+    kvlen[b] = kv_len(P, b, &fl);
+    if (P->layout_kv == ORACLE_PA_BBND)
+      kvstored[b] = ceil_div(kvlen[b], P->page_size) * P->page_size;
+    else
+      kvstored[b] = kv_stored(P, b, &fl);
+  }
+  if (flags) *flags |= fl;
+  return 0;
+}
+
 /* ============================================================ flag scan */
 /* Every status bit the inputs raise: each existing index row, each length,
  * each block-table slot covering a used kv token. */
