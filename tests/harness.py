@@ -8,18 +8,19 @@ import torch
 import block_sparse_variable_b200 as bsa
 
 # Parity criteria for bf16/fp16 inputs: max-abs 2e-2 and rel-L2 1e-2 for
-# out/dq/dk/dv, 1e-3 absolute for lse.  The absolute bound is read as a bound
-# for unit-scale entries: an entry with |ref| > 1 may differ by 2e-2*|ref|
-# (a bf16 result of magnitude 51 already carries a rounding error of up to
-# 0.1, so no bf16 output could meet a flat 2e-2 there).
+# out/dq/dk/dv, 1e-3 absolute for lse.  out (a convex combination of V rows,
+# |out| < ~6 for N(0,1) data) is held to the literal absolute bound.  For
+# dq/dk/dv the absolute bound is read as a bound for unit-scale entries: an
+# entry with |ref| > 1 may differ by 2e-2*|ref| (a bf16 gradient of magnitude
+# 51 already carries a rounding error of up to 0.1, so no bf16 output could
+# meet a flat 2e-2 there); their literal max-abs and the count of entries
+# above 2e-2 are reported (PARITY lines, visible with pytest -s).
 OUT_MAX_ABS = 2e-2
 OUT_REL_L2 = 1e-2
 LSE_ABS = 1e-3
 
 
-def params_of(p, return_lse=True) -> bsa.Params:
-    return bsa.params_for(p.layout_q, p.layout_kv, p.N1, p.N2, (p.BQ, p.BKV), p.scale, return_lse,
-                          getattr(p, "causal", False), getattr(p, "deterministic", False))
+params_of = bsa.params_of_problem
 
 
 def device_inputs(p, device="cuda"):
@@ -55,17 +56,27 @@ def region(ws: torch.Tensor, reg, dtype, count=None) -> np.ndarray:
     return (a if count is None else a[:count]).numpy()
 
 
-def check_close(name, got: torch.Tensor, ref: torch.Tensor, mask=None):
+def check_close(name, got: torch.Tensor, ref: torch.Tensor, mask=None, literal=None):
+    """max-abs and rel-L2 against the oracle.  literal (default: for names
+    starting with "out") applies the flat 2e-2 absolute bound; otherwise the
+    bound scales with |ref| above 1.  Prints one PARITY line with the literal
+    max-abs, the scaled max-abs, rel-L2 and the count of entries above 2e-2."""
     g = got.double().cpu()
     r = ref.double().cpu()
     if mask is not None:
         g, r = g[mask], r[mask]
     assert torch.isfinite(g).all(), f"{name}: non-finite values"
+    if literal is None:
+        literal = name.startswith("out")
     err = (g - r).abs()
     max_abs = float(err.max()) if err.numel() else 0.0
     scaled = float((err / r.abs().clamp(min=1.0)).max()) if err.numel() else 0.0
+    over = int((err > OUT_MAX_ABS).sum())
     rel = float(torch.linalg.vector_norm(g - r) / max(float(torch.linalg.vector_norm(r)), 1e-30))
-    assert scaled <= OUT_MAX_ABS, \
+    print(f"PARITY {name}: max_abs {max_abs:.3e} scaled {scaled:.3e} rel_l2 {rel:.3e} "
+          f"over_2e-2 {over}/{err.numel()} max_ref {float(r.abs().max()) if r.numel() else 0.0:.3e}")
+    bound = max_abs if literal else scaled
+    assert bound <= OUT_MAX_ABS, \
         f"{name}: max-abs {max_abs:.3e}, scaled {scaled:.3e} (max|ref| {float(r.abs().max()):.3e})"
     assert rel <= OUT_REL_L2, f"{name}: rel-L2 {rel:.3e}"
     return max_abs, rel
@@ -84,23 +95,46 @@ def check_lse(got: torch.Tensor, ref: torch.Tensor, mask=None):
         assert err <= LSE_ABS, f"lse: max-abs {err:.3e}"
 
 
-def kv_written_mask(p) -> torch.Tensor:
-    """Rows of dk/dv the backward writes (every stored row of every batch;
-    under paging, the rows of the pages covering each batch's used length)."""
-    shape = p.k.shape[:-1]
-    if p.layout_kv != "PA_BBND":
-        m = torch.zeros(shape, dtype=torch.bool)
-        if p.layout_kv == "BNSD":
-            m[:] = True
-        else:
-            m[:int(p.cu_kv[-1])] = True
-        return m
-    m = torch.zeros(shape, dtype=torch.bool)
-    lens = p.seqused_kv.tolist()
+def q_defined_mask(p) -> torch.Tensor:
+    """Rows of the q-layout tensors (out, lse, dq) that belong to a batch:
+    every row for BNSD; for TND the rows cu_seqlens_q[b] .. + qlen_b of each
+    batch whose lengths are consistent (the oracle's reading of the lengths;
+    rows of no batch are not written)."""
+    import oracle
+    if p.layout_q == "BNSD":
+        return torch.ones(p.q.shape[:-1], dtype=torch.bool)
+    qlen = oracle.Oracle(p).batch_lengths()[0]
+    m = torch.zeros(p.q.shape[:-1], dtype=torch.bool)
     for b in range(p.B):
-        n = -(-lens[b] // p.page_size)
+        a = int(p.cu_q[b])
+        m[a:a + qlen[b]] = True
+    return m
+
+
+def kv_written_mask(p) -> torch.Tensor:
+    """Rows of dk/dv the backward writes: every stored row of every batch
+    whose lengths are consistent (zeros past the used length); under paging,
+    the rows of the pages that the table entries covering each batch's used
+    length name (an entry outside the page range names no page)."""
+    import oracle
+    shape = p.k.shape[:-1]
+    m = torch.zeros(shape, dtype=torch.bool)
+    if p.layout_kv == "BNSD":
+        m[:] = True
+        return m
+    _, kvlen, kvst, _ = oracle.Oracle(p).batch_lengths()
+    if p.layout_kv == "TND":
+        for b in range(p.B):
+            a = int(p.cu_kv[b])
+            m[a:a + kvst[b]] = True
+        return m
+    P = int(p.k.shape[0])
+    for b in range(p.B):
+        n = -(-kvlen[b] // p.page_size)
         for x in range(n):
-            m[int(p.block_table[b, x])] = True
+            pg = int(p.block_table[b, x])
+            if 0 <= pg < P:
+                m[pg] = True
     return m
 
 
