@@ -12,6 +12,8 @@
 //     sort of 4096-key chunks followed by a merge by rank.
 #include <cuda_runtime.h>
 
+#include <cmath>
+
 #include "bsa_internal.h"
 
 namespace bsa {
@@ -21,6 +23,7 @@ __device__ __forceinline__ int64_t cdiv64(int64_t a, int64_t b) { return (a + b 
 
 __global__ void k_geometry(Problem p) {
   __shared__ uint32_t sflags;
+  __shared__ int64_t s_sum_nq;
   uint32_t *st = p.status;
   for (int i = threadIdx.x; i < kStWords; i += blockDim.x) st[i] = 0;
   for (int64_t r = threadIdx.x; r < p.Rg; r += blockDim.x) p.row_batch[r] = -1;
@@ -50,6 +53,15 @@ __global__ void k_geometry(Problem p) {
       const int64_t u = p.seqused_kv[b];
       if (u < 0 || u > kvst) { f |= BSA_FLAG_BAD_SEQLEN; kvlen = 0; }
       else kvlen = u;
+    }
+    if (p.kv_layout == BSA_LAYOUT_PA_BBND) {
+      // every table entry that covers a used kv token must name a page; the
+      // tokens of a bad entry take no part (whether or not a row selects them)
+      const int64_t used = cdiv64(kvlen, p.page_size);
+      for (int64_t x = 0; x < used; ++x) {
+        const int32_t pg = p.block_table[int64_t(b) * p.bt_s0 + x];
+        if (pg < 0 || pg >= p.num_pages) f |= BSA_FLAG_BAD_PAGE;
+      }
     }
     BatchInfo bi;
     bi.qlen = int32_t(qlen);
@@ -89,9 +101,42 @@ __global__ void k_geometry(Problem p) {
     if (p.q_layout == BSA_LAYOUT_TND && qo > p.R) f |= BSA_FLAG_BAD_INDEX;
     st[kStTK] = uint32_t(ko);
     st[kStSumNq] = uint32_t(qo);
+    s_sum_nq = qo;
     if (f) atomicOr(&sflags, f);
   }
   __syncthreads();
+
+  // Query blocks past the last index row (TND, an index with fewer rows than
+  // the lengths need) select nothing: their rows get out 0 and lse -inf in
+  // the forward, dq 0 in the deterministic backward (whose dq pass visits
+  // work items only; the default backward converts every accumulator row).
+  const bool fwd = p.dq == nullptr;
+  if (s_sum_nq > p.R && (fwd || p.deterministic)) {
+    const int CH = p.D / 8;  // 16-byte chunks of a 16-bit row
+    for (int b = 0; b < p.B; ++b) {
+      const BatchInfo bi = p.batch[b];
+      const int64_t i0 = p.R - bi.qoff > 0 ? p.R - bi.qoff : 0;
+      const int64_t t0 = i0 * p.BQ;
+      const int64_t nrow = bi.qlen > t0 ? bi.qlen - t0 : 0;
+      for (int64_t x = threadIdx.x; x < nrow * p.N1 * CH; x += blockDim.x) {
+        const int ch = int(x % CH);
+        const int h = int((x / CH) % p.N1);
+        const int t = int(t0 + x / (int64_t(CH) * p.N1));
+        const uint4 z = make_uint4(0, 0, 0, 0);
+        if (fwd) {
+          uint16_t *o = static_cast<uint16_t *>(p.out) + int64_t(b) * p.o_sb +
+                        (bi.q_tok0 + t) * p.o_st + int64_t(h) * p.o_sh;
+          reinterpret_cast<uint4 *>(o)[ch] = z;
+          if (ch == 0 && p.lse)
+            p.lse[int64_t(b) * p.l_sb + (bi.q_tok0 + t) * p.l_st + int64_t(h) * p.l_sh] = -INFINITY;
+        } else {
+          uint16_t *o = static_cast<uint16_t *>(p.dq) + int64_t(b) * p.dq_sb +
+                        (bi.q_tok0 + t) * p.dq_st + int64_t(h) * p.dq_sh;
+          reinterpret_cast<uint4 *>(o)[ch] = z;
+        }
+      }
+    }
+  }
 
   for (int b = threadIdx.x; b < p.B; b += blockDim.x) {
     const BatchInfo bi = p.batch[b];

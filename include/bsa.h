@@ -35,7 +35,23 @@
  * *values* of cu_seqlens, seqused_kv, the index and the block table are not
  * read on the host (GenericBlockSparseAttention article, "values are not
  * checked at tiling").  The device skips invalid values and records them as
- * BSA_FLAG_* bits in the workspace status word, read with bsa_read_status.
+ * BSA_FLAG_* bits in the workspace status word, read with bsa_read_status;
+ * no invalid value is used as an address.  The readings (the pages leave
+ * them open):
+ *   - a cu_seqlens pair that decreases, starts below 0 or ends past its
+ *     tensor, or a seqused_kv below 0 or above the stored kv length, counts
+ *     as length 0 (BAD_SEQLEN): a query batch without rows, a kv batch
+ *     nothing can select (its index entries are then out of range:
+ *     BAD_INDEX).  Batches whose ranges overlap (possible only with a
+ *     decreasing cu_seqlens) give unspecified results for the shared rows;
+ *   - a block-table entry outside [0, num_pages) that covers a used kv token
+ *     raises BAD_PAGE, whether or not a row selects it; the tokens it covers
+ *     take no part, and the backward writes no dk/dv for them;
+ *   - a TND query block with no index row (fewer rows than the lengths need)
+ *     selects nothing (BAD_INDEX): out 0, lse -inf, dq 0.
+ * Rows of the q-layout tensors that belong to no batch (past the last
+ * batch, or of a batch whose cu_seqlens_q pair is invalid) are not written
+ * by the forward; the default backward writes dq 0 there.
  */
 #ifndef BSA_H_
 #define BSA_H_
@@ -112,10 +128,13 @@ typedef enum bsa_status {
 } bsa_status;
 
 /* Bits of the device status word (bsa_read_status). */
-#define BSA_FLAG_BAD_INDEX 0x1u   /* an index entry >= ceil(kvlen/BKV), not ascending,
-                                     or more query blocks than index rows (TND) */
-#define BSA_FLAG_BAD_SEQLEN 0x2u  /* cu_seqlens / seqused_kv contradict the storage */
-#define BSA_FLAG_BAD_PAGE 0x4u    /* a block-table entry outside [0, num_pages) */
+#define BSA_FLAG_BAD_INDEX 0x1u   /* an index entry >= ceil(kvlen/BKV) or not above the
+                                     previous accepted entry (skipped), or more query
+                                     blocks than index rows (TND) */
+#define BSA_FLAG_BAD_SEQLEN 0x2u  /* cu_seqlens / seqused_kv contradict the storage
+                                     (that length counts as 0) */
+#define BSA_FLAG_BAD_PAGE 0x4u    /* a block-table entry outside [0, num_pages) covers
+                                     a used kv token (its tokens take no part) */
 #define BSA_FLAG_TIMEOUT 0x8u     /* a bounded device wait gave up (pipeline fault) */
 #define BSA_FLAG_INTERNAL 0x10u   /* a kernel precondition failed (internal error) */
 
@@ -135,9 +154,9 @@ typedef enum bsa_status {
  *   seqused_kv     I32 [B], optional; required for PA_BBND.  kv tokens at or
  *                  past seqused_kv[b] are ignored.
  *   block_table    I32 [B, max_pages], required for PA_BBND
- *   out     same shape/dtype as q (written for every q row; rows with no
- *           selected key get 0); F16 or BF16 for F8E4M3 inputs, and then
- *           its dtype is the output type
+ *   out     same shape/dtype as q (written for every query row of every
+ *           batch; rows with no selected key get 0); F16 or BF16 for F8E4M3
+ *           inputs, and then its dtype is the output type
  *   lse     F32, BNSD [B,N1,Sq] / TND [Tq,N1]; required when return_lse
  *           (rows with no selected key get -inf)
  * FP8 inputs (GenericBlockSparseAttention article, quantization table,
@@ -178,9 +197,12 @@ bsa_status bsa_fwd(const bsa_tensor *q, const bsa_tensor *k, const bsa_tensor *v
  * loading the library keeps until the process exits.
  *   - A problem whose forward workspace (bsa_fwd_get_workspace) exceeds
  *     32 MiB is rejected with BSA_ERR_WORKSPACE before any launch.
- *   - The first call on a device looks up the array's device address
- *     (a CUDA runtime query) and caches it; make that first call before any
- *     stream capture on that device.
+ *   - The first call on a device sets the array up there: CUDA places a
+ *     module's device data on the GPU when it is first used, so that call
+ *     grows device memory by the 32 MiB, then looks the array's address up
+ *     and caches it.  Make one call per device at start-up -- before the
+ *     phase in which the caller may not allocate, and before any stream
+ *     capture on that device; later calls allocate nothing.
  *   - All calls share the one array, which keeps the last call's contents;
  *     each call initialises everything it reads, but two calls that may
  *     overlap on the GPU (different streams, different threads) race and
@@ -298,9 +320,9 @@ bsa_status bsa_bwd_workspace_layout(const bsa_tensor *q, const bsa_tensor *k, co
 bsa_status bsa_set_main_kernel_events(void *before, void *after);
 
 /* Diagnostic (the pages have no counterpart).  For n floats x (device
- * memory), writes y_poly[i] = the FMA-pipe 2^x the softmax kernels use for part
- * of their exponentials (range reduction plus a degree-3 minimax polynomial,
- * relative error <= 7.5e-5 for x >= -126) and y_mufu[i] = the hardware
+ * memory), writes y_poly[i] = an FMA-pipe 2^x (range reduction plus a degree-3
+ * minimax polynomial, relative error <= 7.5e-5 for -126 <= x < 128, +inf from
+ * 128 up; a building block no shipped kernel calls) and y_mufu[i] = the hardware
  * ex2.approx of x, asynchronously on `stream`.  Caller-owned device buffers;
  * BSA_ERR_NULLPTR for a NULL buffer with n > 0, BSA_ERR_PARAM_INVALID for
  * n < 0, BSA_ERR_CUDA if the launch fails. */
