@@ -282,7 +282,6 @@ def job_tflops(world, flops_per_replica_step, ms_per_step):
 def run_ours(args):
     import block_sparse_variable_b200 as bsa
     import workloads
-    from tests.harness import params_of
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -301,7 +300,7 @@ def run_ours(args):
     p = workloads.make_config(args.config, args.batch, args.causal)
     p.deterministic = args.deterministic
     pairs = _pairs(p)
-    P = params_of(p)
+    P = bsa.params_of_problem(p)
     to = lambda t: None if t is None else t.to(dev)  # noqa: E731
     q, k, v, dout, index = (to(getattr(p, n)) for n in ("q", "k", "v", "dout", "index"))
     opt = dict(cu_seqlens_q=to(p.cu_q), cu_seqlens_kv=to(p.cu_kv), seqused_kv=to(p.seqused_kv),
@@ -448,7 +447,6 @@ def run_fp8(args):
     bf16 burst x 2 (the nominal fp8 / bf16 tensor ratio, 4.5 / 2.25 PFLOP/s)."""
     import block_sparse_variable_b200 as bsa
     import workloads
-    from tests.harness import params_of
 
     if int(os.environ.get("WORLD_SIZE", "1")) > 1:
         raise SystemExit("--fp8 is a one-GPU line; run it without torchrun")
@@ -456,7 +454,7 @@ def run_fp8(args):
     dev = torch.device("cuda", 0)
     p = workloads.make_config(3, fp8=True)
     pairs = _pairs(p)
-    P = params_of(p)
+    P = bsa.params_of_problem(p)
     q, k, v, index = (getattr(p, n).to(dev) for n in ("q", "k", "v", "index"))
     out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)

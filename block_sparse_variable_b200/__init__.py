@@ -187,6 +187,15 @@ def params_for(q_layout, kv_layout, num_heads, num_kv_heads=0, block_shape=(128,
                   bool(causal), bool(deterministic))
 
 
+def params_of_problem(prob, return_lse=True) -> Params:
+    """Params for a problem description: any object with the attributes
+    layout_q, layout_kv, N1, N2, BQ, BKV, scale and, optionally, causal and
+    deterministic (for example a ``workloads.Problem``)."""
+    return params_for(prob.layout_q, prob.layout_kv, prob.N1, prob.N2, (prob.BQ, prob.BKV),
+                      prob.scale, return_lse, getattr(prob, "causal", False),
+                      getattr(prob, "deterministic", False))
+
+
 def _fwd_descs(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table, out, lse):
     return [describe(x) for x in (q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv,
                                   block_table)], describe(out), describe(lse)

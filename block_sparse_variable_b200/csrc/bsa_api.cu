@@ -355,6 +355,17 @@ void take_events(cudaEvent_t &before, cudaEvent_t &after) {
   t_ev_before = t_ev_after = nullptr;
 }
 
+}  // namespace
+
+namespace bsa {
+void drop_pending_events() {
+  cudaEvent_t a, b;
+  take_events(a, b);
+}
+}  // namespace bsa
+
+namespace {
+
 bsa_status run_fwd(const Problem &p, cudaStream_t s, cudaEvent_t e0, cudaEvent_t e1) {
   BSA_LAUNCH(bsa::launch_prep_geometry(p, s));
   BSA_LAUNCH(bsa::launch_prep_compact(p, true, s));

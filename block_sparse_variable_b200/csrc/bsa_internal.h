@@ -101,4 +101,9 @@ cudaError_t launch_dq_main(const Problem &p, cudaStream_t s);
 
 int num_sms();
 
+// clears the event pair bsa_set_main_kernel_events armed for this host
+// thread's next call (for entry points that return before reaching bsa_fwd
+// or bsa_bwd, which consume it)
+void drop_pending_events();
+
 }  // namespace bsa

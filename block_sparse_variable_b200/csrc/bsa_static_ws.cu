@@ -12,7 +12,10 @@
 // name as an address: the host-side name is only a stand-in, and a kernel
 // given it would fault or, where the GPU can reach host memory, silently
 // use the wrong memory.  The device address is looked up once per device
-// with cudaGetSymbolAddress and cached.
+// with cudaGetSymbolAddress and cached.  CUDA places the array on a device
+// when this file's module is first used there, i.e. at that first lookup: the
+// first call on each device grows device memory by the array's size, later
+// calls allocate nothing.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -58,10 +61,13 @@ bsa_status bsa_fwd_static_workspace(const bsa_tensor *q, const bsa_tensor *k, co
   size_t need = 0;
   bsa_status st = bsa_fwd_get_workspace(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv,
                                         block_table, params, out, lse, &need);
-  if (st != BSA_OK) return st;
-  if (need > kStaticScratchBytes) return BSA_ERR_WORKSPACE;
+  if (st == BSA_OK && need > kStaticScratchBytes) st = BSA_ERR_WORKSPACE;
   void *scratch = nullptr;
-  if ((st = scratch_address(&scratch)) != BSA_OK) return st;
+  if (st == BSA_OK) st = scratch_address(&scratch);
+  if (st != BSA_OK) {
+    bsa::drop_pending_events();  // a pair armed for this call ends with it
+    return st;
+  }
   return bsa_fwd(q, k, v, index, cu_seqlens_q, cu_seqlens_kv, seqused_kv, block_table, params, out,
                  lse, scratch, kStaticScratchBytes, stream);
 }

@@ -11,7 +11,7 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
-#include "ptx_sm80.cuh"
+#include "pack16.cuh"
 
 namespace bsa {
 namespace {
@@ -35,8 +35,8 @@ __global__ void k_bwd_pre(const Problem p) {
   const T *O = static_cast<const T *>(p.out) + qstore_off(p, p.o_sb, p.o_sh, p.o_st, r, h);
   float acc = 0.f;
   for (int d = lane * 2; d < p.D; d += 64) {
-    const float2 a = MmaOp<T>::unpack(*reinterpret_cast<const uint32_t *>(dO + d));
-    const float2 c = MmaOp<T>::unpack(*reinterpret_cast<const uint32_t *>(O + d));
+    const float2 a = Pack2<T>::unpack(*reinterpret_cast<const uint32_t *>(dO + d));
+    const float2 c = Pack2<T>::unpack(*reinterpret_cast<const uint32_t *>(O + d));
     acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
   }
 #pragma unroll
@@ -57,10 +57,10 @@ __global__ void k_dq_convert(const Problem p) {
   const float4 x0 = *reinterpret_cast<const float4 *>(p.dq_acc + e);
   const float4 x1 = *reinterpret_cast<const float4 *>(p.dq_acc + e + 4);
   uint4 o;
-  o.x = MmaOp<T>::pack(x0.x * p.scale, x0.y * p.scale);
-  o.y = MmaOp<T>::pack(x0.z * p.scale, x0.w * p.scale);
-  o.z = MmaOp<T>::pack(x1.x * p.scale, x1.y * p.scale);
-  o.w = MmaOp<T>::pack(x1.z * p.scale, x1.w * p.scale);
+  o.x = Pack2<T>::pack(x0.x * p.scale, x0.y * p.scale);
+  o.y = Pack2<T>::pack(x0.z * p.scale, x0.w * p.scale);
+  o.z = Pack2<T>::pack(x1.x * p.scale, x1.y * p.scale);
+  o.w = Pack2<T>::pack(x1.z * p.scale, x1.w * p.scale);
   *reinterpret_cast<uint4 *>(static_cast<T *>(p.dq) + qstore_off(p, p.dq_sb, p.dq_sh, p.dq_st, r, h) +
                              d) = o;
 }

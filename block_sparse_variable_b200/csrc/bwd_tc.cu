@@ -39,7 +39,7 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
-#include "ptx_sm80.cuh"
+#include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
 #include "tc_device.cuh"
@@ -462,8 +462,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
               }
               const float s0 = p0 * (__uint_as_float(bd[c2]) - dsum[q]);
               const float s1 = p1 * (__uint_as_float(bd[c2 + 1]) - dsum[q + 1]);
-              pp[8 * k + (c2 >> 1)] = MmaOp<T>::pack(p0, p1);
-              dd[8 * k + (c2 >> 1)] = MmaOp<T>::pack(s0, s1);
+              pp[8 * k + (c2 >> 1)] = Pack2<T>::pack(p0, p1);
+              dd[8 * k + (c2 >> 1)] = Pack2<T>::pack(s0, s1);
             }
             if (k + 1 < 4) tmem_wait_ld();
           }
@@ -554,14 +554,14 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
             for (int c = 0; c < 32; c += 8) {
               uint4 wk, wv;
-              wk.x = MmaOp<T>::pack(__uint_as_float(xk[c]) * p.scale, __uint_as_float(xk[c + 1]) * p.scale);
-              wk.y = MmaOp<T>::pack(__uint_as_float(xk[c + 2]) * p.scale, __uint_as_float(xk[c + 3]) * p.scale);
-              wk.z = MmaOp<T>::pack(__uint_as_float(xk[c + 4]) * p.scale, __uint_as_float(xk[c + 5]) * p.scale);
-              wk.w = MmaOp<T>::pack(__uint_as_float(xk[c + 6]) * p.scale, __uint_as_float(xk[c + 7]) * p.scale);
-              wv.x = MmaOp<T>::pack(__uint_as_float(xv[c]), __uint_as_float(xv[c + 1]));
-              wv.y = MmaOp<T>::pack(__uint_as_float(xv[c + 2]), __uint_as_float(xv[c + 3]));
-              wv.z = MmaOp<T>::pack(__uint_as_float(xv[c + 4]), __uint_as_float(xv[c + 5]));
-              wv.w = MmaOp<T>::pack(__uint_as_float(xv[c + 6]), __uint_as_float(xv[c + 7]));
+              wk.x = Pack2<T>::pack(__uint_as_float(xk[c]) * p.scale, __uint_as_float(xk[c + 1]) * p.scale);
+              wk.y = Pack2<T>::pack(__uint_as_float(xk[c + 2]) * p.scale, __uint_as_float(xk[c + 3]) * p.scale);
+              wk.z = Pack2<T>::pack(__uint_as_float(xk[c + 4]) * p.scale, __uint_as_float(xk[c + 5]) * p.scale);
+              wk.w = Pack2<T>::pack(__uint_as_float(xk[c + 6]) * p.scale, __uint_as_float(xk[c + 7]) * p.scale);
+              wv.x = Pack2<T>::pack(__uint_as_float(xv[c]), __uint_as_float(xv[c + 1]));
+              wv.y = Pack2<T>::pack(__uint_as_float(xv[c + 2]), __uint_as_float(xv[c + 3]));
+              wv.z = Pack2<T>::pack(__uint_as_float(xv[c + 4]), __uint_as_float(xv[c + 5]));
+              wv.w = Pack2<T>::pack(__uint_as_float(xv[c + 6]), __uint_as_float(xv[c + 7]));
               *reinterpret_cast<uint4 *>(dkr + c) = wk;
               *reinterpret_cast<uint4 *>(dvr + c) = wv;
             }

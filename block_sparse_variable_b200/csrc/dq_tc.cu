@@ -38,7 +38,7 @@
 #include "coalesce.cuh"
 #include "bsa_internal.h"
 #include "fwd_walk.cuh"
-#include "ptx_sm80.cuh"
+#include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
 #include "tc_device.cuh"
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kDThreads, 1)
                 s0 = c < valid ? s0 : 0.f;
                 s1 = c + 1 < valid ? s1 : 0.f;
               }
-              dd[8 * k + (c2 >> 1)] = MmaOp<T>::pack(s0, s1);
+              dd[8 * k + (c2 >> 1)] = Pack2<T>::pack(s0, s1);
             }
             if (k + 1 < 4) tmem_wait_ld();
           }
@@ -386,10 +386,10 @@ __global__ void __launch_bounds__(kDThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
-            qch[4 * h + c].x = MmaOp<T>::pack(__uint_as_float(x[8 * c]) * p.scale, __uint_as_float(x[8 * c + 1]) * p.scale);
-            qch[4 * h + c].y = MmaOp<T>::pack(__uint_as_float(x[8 * c + 2]) * p.scale, __uint_as_float(x[8 * c + 3]) * p.scale);
-            qch[4 * h + c].z = MmaOp<T>::pack(__uint_as_float(x[8 * c + 4]) * p.scale, __uint_as_float(x[8 * c + 5]) * p.scale);
-            qch[4 * h + c].w = MmaOp<T>::pack(__uint_as_float(x[8 * c + 6]) * p.scale, __uint_as_float(x[8 * c + 7]) * p.scale);
+            qch[4 * h + c].x = Pack2<T>::pack(__uint_as_float(x[8 * c]) * p.scale, __uint_as_float(x[8 * c + 1]) * p.scale);
+            qch[4 * h + c].y = Pack2<T>::pack(__uint_as_float(x[8 * c + 2]) * p.scale, __uint_as_float(x[8 * c + 3]) * p.scale);
+            qch[4 * h + c].z = Pack2<T>::pack(__uint_as_float(x[8 * c + 4]) * p.scale, __uint_as_float(x[8 * c + 5]) * p.scale);
+            qch[4 * h + c].w = Pack2<T>::pack(__uint_as_float(x[8 * c + 6]) * p.scale, __uint_as_float(x[8 * c + 7]) * p.scale);
           }
         }
       } else {

@@ -1,5 +1,8 @@
-// exp2_poly.cuh -- 2^x on the FMA pipe, to share the softmax exponentials
-// between the MUFU unit (ex2.approx) and the FP32 pipe.
+// exp2_poly.cuh -- 2^x on the FMA pipe: a building block for sharing softmax
+// exponentials between the MUFU unit (ex2.approx) and the FP32 pipe.  No
+// shipped kernel calls it (measured: the softmax warps are issue-bound, so
+// moving exponentials to the FMA pipe made the forward slower); it is kept
+// with its device self test (bsa_selftest_exp2).
 //
 // x = n + f with n = round(x) (by adding 1.5 * 2^23, which leaves n in the
 // low mantissa bits) and |f| <= 1/2; 2^f = p(f) with p the degree-3
@@ -8,7 +11,9 @@
 // error 7.5e-5 in fp32 Horner evaluation); 2^n is added into the exponent
 // field.  x is clamped at -126 so that the exponent field stays >= 0: below
 // that the result is a positive number under 2^-125 instead of the exact
-// value (every use here treats such a value as zero).
+// value (every use here treats such a value as zero).  x >= 128 gives +inf,
+// as the hardware exponential does (the exponent field would otherwise run
+// into the sign bit and give a wrong finite value or a NaN).
 #pragma once
 
 namespace bsa {
@@ -25,7 +30,8 @@ __device__ __forceinline__ float exp2_poly(float x) {
   float p = fmaf(kExp2C3, f, kExp2C2);
   p = fmaf(p, f, kExp2C1);
   p = fmaf(p, f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  const float y = __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  return x >= 128.0f ? __int_as_float(0x7f800000) : y;
 }
 
 }  // namespace bsa

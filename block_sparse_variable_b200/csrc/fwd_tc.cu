@@ -39,10 +39,9 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
-#include "exp2_poly.cuh"
 #include "fp8.cuh"
 #include "fwd_walk.cuh"
-#include "ptx_sm80.cuh"
+#include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
 #include "tc_device.cuh"
@@ -65,9 +64,6 @@ constexpr int kCols = 128 / kSoftmaxGroups;  // kv columns per softmax thread
 // a row takes a new reference max once its P could exceed 2^8 (a half-row
 // sum of P above 2^8)
 constexpr float kRescaleSum = 256.0f;
-// of every 8 column pairs, this many take their exponentials on the FMA pipe
-// (exp2_poly) instead of the MUFU unit, which alone would bound the softmax
-constexpr int kPolyPairsOf8 = 0;
 
 // barrier slots
 enum : int {
@@ -384,9 +380,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             for (int c = 0; c < kCols; c += 2) {
               const float a0 = fmaf(__uint_as_float(x[c]), p.scale_log2, -mm);
               const float a1 = fmaf(__uint_as_float(x[c + 1]), p.scale_log2, -mm);
-              const bool poly = ((c >> 1) & 7) < kPolyPairsOf8;  // fixed per unrolled c
-              const float e0 = poly ? exp2_poly(a0) : ex2(a0);
-              const float e1 = poly ? exp2_poly(a1) : ex2(a1);
+              const float e0 = ex2(a0);
+              const float e1 = ex2(a1);
               ps[(c >> 1) & 1] += e0 + e1;
               if constexpr (kFp8) {
                 // P in e4m3, four to a 32-bit column (the pair before is in
@@ -394,7 +389,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 if ((c & 2) == 0) pk[c >> 2] = __float_as_uint(e0), pk[(c >> 2) + kCols / 4] = __float_as_uint(e1);
                 else pk[c >> 2] = pack_e4m3x4(__uint_as_float(pk[c >> 2]), __uint_as_float(pk[(c >> 2) + kCols / 4]), e0, e1);
               } else {
-                pk[c >> 1] = MmaOp<T>::pack(e0, e1);
+                pk[c >> 1] = Pack2<T>::pack(e0, e1);
               }
             }
           };
@@ -512,10 +507,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int c8 = 0; c8 < kOc / 8; ++c8) {
             uint4 w;
-            w.x = MmaOp<T>::pack(__uint_as_float(o[8 * c8]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
-            w.y = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
-            w.z = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
-            w.w = MmaOp<T>::pack(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
+            w.x = Pack2<T>::pack(__uint_as_float(o[8 * c8]) * inv, __uint_as_float(o[8 * c8 + 1]) * inv);
+            w.y = Pack2<T>::pack(__uint_as_float(o[8 * c8 + 2]) * inv, __uint_as_float(o[8 * c8 + 3]) * inv);
+            w.z = Pack2<T>::pack(__uint_as_float(o[8 * c8 + 4]) * inv, __uint_as_float(o[8 * c8 + 5]) * inv);
+            w.w = Pack2<T>::pack(__uint_as_float(o[8 * c8 + 6]) * inv, __uint_as_float(o[8 * c8 + 7]) * inv);
             reinterpret_cast<uint4 *>(orow + wg * kOc)[c8] = w;
           }
         }

@@ -5,7 +5,7 @@
 #include "bsa_internal.h"
 #include "exp2_poly.cuh"
 #include "fp8.cuh"
-#include "ptx_sm80.cuh"
+#include "pack16.cuh"
 #include "tc_device.cuh"
 
 namespace bsa {

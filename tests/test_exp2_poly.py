@@ -1,5 +1,5 @@
-"""The FMA-pipe 2^x that the softmax kernels use for part of their
-exponentials (csrc/exp2_poly.cuh).
+"""The FMA-pipe 2^x building block (csrc/exp2_poly.cuh), which no shipped
+kernel calls; it is kept with its device self test.
 
 CPU: the header's coefficients are the ones the Remez fit in csrc/exp2_fit.py
 derives, and a bit-exact numpy model of the device routine (same fp32
@@ -42,7 +42,7 @@ def _model(x):
     p = (p * f + c[1]).astype(np.float32)     # the model's error is a slight upper bound
     p = (p * f + c[0]).astype(np.float32)
     bits = p.view(np.int32) + (t.view(np.int32) << np.int32(23))
-    return bits.view(np.float32)
+    return np.where(x >= np.float32(128.0), np.float32(np.inf), bits.view(np.float32))
 
 
 def test_header_coefficients_are_the_remez_fit():
@@ -61,6 +61,17 @@ def test_model_relative_error_over_the_softmax_range():
     assert float(rel.max()) <= BOUND + 2e-7  # + the model's extra fp32 roundings
     # exact powers of two of the integer part: 2^n * p(0)
     assert _model(np.float32([3.0]))[0] == np.float32(8.0 * np.float32(_header_coefficients()[0]))
+
+
+def test_model_overflow_is_inf_and_top_range_is_accurate():
+    """x >= 128 overflows to +inf (as the hardware exponential does); just
+    below, the exponent field still holds the exact power of two."""
+    with np.errstate(over="ignore"):
+        y = _model(np.float32([128.0, 128.5, 200.0, np.inf]))
+    assert np.all(np.isposinf(y))
+    x = np.linspace(120.0, 127.99, 10001, dtype=np.float32)
+    rel = np.abs(_model(x).astype(np.float64) / np.exp2(x.astype(np.float64)) - 1)
+    assert float(rel.max()) <= BOUND + 2e-7
 
 
 def test_model_underflow_is_tiny_and_positive():
@@ -87,3 +98,6 @@ def test_device_exp2_poly_against_exact_and_mufu():
     torch.cuda.synchronize()
     assert bool((tails[0] > 0).all()) and bool((tails[0] < 2.0 ** -125).all())
     assert float(tails[1][2]) == 0.0
+    top = bsa.bsa_selftest_exp2(torch.tensor([127.9, 128.0, 129.5, math.inf], device="cuda"))
+    torch.cuda.synchronize()
+    assert math.isfinite(float(top[0][0])) and bool(torch.isposinf(top[0][1:]).all())
