@@ -96,6 +96,36 @@ def _pairs(p):
     return total
 
 
+def _alg_bytes(p):
+    """Algorithmic bytes of one forward and one backward call: every tensor
+    the pass must touch, once.  Forward: Q, out, lse, the index and the K, V
+    rows of the kv blocks some row of the kv head's group selects.  Backward:
+    Q, out, dOut, lse read and dQ written; those K, V rows read; dK, dV
+    written for every used kv row (zeros where nothing selects it)."""
+    es = 1 if p.dtype == torch.float8_e4m3fn else 2
+    D, N1, N2 = p.D, p.N1, p.N2
+    g = N1 // N2
+    tq = sum(p.lens_q) if p.layout_q == "TND" else p.B * p.q.shape[2]
+    qb = tq * N1 * D
+    idx = p.index.view(torch.int16).numpy().view(np.uint16).astype(np.int64)
+    kv_sel = 0   # selected kv rows, summed over kv heads
+    off = 0
+    for b in range(p.B):
+        nq = -(-p.lens_q[b] // p.BQ)
+        for h2 in range(N2):
+            his = range(h2 * g, (h2 + 1) * g) if p.Hidx == N1 else [h2]
+            rows = [idx[b, hi, :nq] if p.layout_q == "BNSD" else idx[hi, off:off + nq] for hi in his]
+            blocks = set(int(x) for r in rows for x in r.ravel()) - {0xFFFF}
+            kv_sel += sum(max(0, min(p.BKV, p.lens_kv[b] - j * p.BKV)) for j in blocks)
+        off += nq if p.layout_q == "TND" else 0
+    kv_used = sum(p.lens_kv) * N2
+    small = p.index.numel() * 2 + sum(0 if t is None else t.numel() * t.element_size()
+                                      for t in (p.cu_q, p.cu_kv, p.seqused_kv, p.block_table))
+    fwd = qb * es + qb * 2 + tq * N1 * 4 + 2 * kv_sel * D * es + small
+    bwd = qb * 2 * 4 + tq * N1 * 4 + 2 * kv_sel * D * 2 + 2 * kv_used * D * 2 + small
+    return fwd, bwd
+
+
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples during the timed region."""
 
@@ -149,16 +179,33 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- oracle leg
-def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = False):
+def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = False,
+                       shared_rows: bool = False):
     """A bounded slice of the workload for the CPU oracle: batch 0, head 0,
     the first q_rows query rows against the full key range (causal: the
     last q_rows rows, which keeps every row's place relative to the end of
-    the kv sequence)."""
+    the kv sequence).  TND workloads: batch 0's first q_rows query rows of
+    head 0 against batch 0's kv rows of kv head 0 (gathered out of the pages
+    for a paged cache: the same rows, stored contiguously)."""
     import workloads
     from workloads.gen import make_problem, pat_dense
-    p = workloads.make_config(cfg, causal=causal, fp8=fp8)
+    p = workloads.make_config(cfg, causal=causal, fp8=fp8, shared_rows=shared_rows)
     if p.layout_q != "BNSD":
-        raise SystemExit("CPU baseline slice is defined for the BNSD workloads")
+        L0, kv0 = p.lens_q[0], p.lens_kv[0]
+        q_rows = max(min(L0, p.BQ), min(L0, (q_rows // p.BQ) * p.BQ))
+        sub = make_problem(layout_q="TND", layout_kv="TND", B=1, N1=1, N2=1, D=p.D,
+                           lens_q=[q_rows], lens_kv=[kv0], BQ=p.BQ, BKV=p.BKV, W=p.W,
+                           pattern=pat_dense, dtype=p.dtype, scale=p.scale)
+        sub.q = p.q[:q_rows, :1].contiguous()
+        sub.dout = p.dout[:q_rows, :1].contiguous()
+        if p.layout_kv == "TND":
+            sub.k, sub.v = (t[:kv0, :1].contiguous() for t in (p.k, p.v))
+        else:
+            pages = p.block_table[0, :-(-kv0 // p.page_size)].long()
+            sub.k, sub.v = (t[pages].reshape(-1, p.N2, p.D)[:kv0, :1].contiguous()
+                            for t in (p.k, p.v))
+        sub.index = p.index[:1, :-(-q_rows // p.BQ)].contiguous()
+        return sub
     S = p.q.shape[2]
     q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
     sub = make_problem(B=1, N1=1, N2=1, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
@@ -184,29 +231,38 @@ def _oracle_step(sub):
     return time.perf_counter() - t
 
 
-def _oracle_rate(cfg: int, target_s: float, causal: bool = False):
+def _oracle_rate(cfg: int, target_s: float, causal: bool = False, shared_rows: bool = False):
     """Calibrate the slice to ~target_s per step; returns (sub, pairs)."""
-    sub = _oracle_subproblem(cfg, 128, causal)
+    sub = _oracle_subproblem(cfg, 128, causal, shared_rows=shared_rows)
     t = _oracle_step(sub)
     rows = int(128 * max(1.0, target_s / max(t, 1e-3)))
-    sub = _oracle_subproblem(cfg, rows, causal)
+    sub = _oracle_subproblem(cfg, rows, causal, shared_rows=shared_rows)
     return sub, _pairs(sub)
 
 
-def _descr(cfg: int, causal: bool, deterministic: bool = False) -> str:
+def _descr(cfg: int, causal: bool, deterministic: bool = False, shared_rows: bool = False,
+           per_head_rows: bool = False) -> str:
     return (DESCR[cfg] + (", causal mask + lower-triangular index" if causal else "")
-            + (", deterministic backward" if deterministic else ""))
+            + (", deterministic backward" if deterministic else "")
+            + (", one index row per GQA group (Hidx = N2; packed forward tiles)"
+               if shared_rows and not per_head_rows else "")
+            + (", the per-group index rows copied to every query head (Hidx = N1)"
+               if per_head_rows else ""))
 
 
-def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False):
-    sub, pairs = _oracle_rate(cfg, target_s, causal)
+def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False, shared_rows: bool = False):
+    sub, pairs = _oracle_rate(cfg, target_s, causal, shared_rows)
     t = _oracle_step(sub)
     flops = 14 * sub.D * pairs
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _omp_threads(), "kind": "oracle",
             "sample": f"fp64 oracle fwd+bwd on batch 0, head 0, {'last' if causal else 'first'} "
-                      f"{sub.q.shape[2]} query rows "
-                      f"x {sub.k.shape[2]} keys of {DESCR[cfg].split(':')[0]} ({pairs} kept pairs, "
+                      f"{_rows_of(sub)} query rows "
+                      f"x {sub.lens_kv[0]} keys of {DESCR[cfg].split(':')[0]} ({pairs} kept pairs, "
                       f"{t:.1f} s)"}
+
+
+def _rows_of(sub):
+    return sub.q.shape[2] if sub.layout_q == "BNSD" else sub.q.shape[0]
 
 
 def _omp_threads():
@@ -235,12 +291,13 @@ def run_reference(args):
         metric, per_pair = "effective TFLOP/s (selected blocks only), FP8 forward", 4
         workload = DESCR[3] + ", q/k/v e4m3 (bf16 out), forward only"
     else:
-        sub, pairs = _oracle_rate(args.config, 2.0, args.causal)
+        sub, pairs = _oracle_rate(args.config, 2.0, args.causal, args.shared_rows)
 
         def one():
             return _oracle_step(sub)
         metric, per_pair = METRIC, 14
-        workload = _descr(args.config, args.causal, getattr(args, "deterministic", False))
+        workload = _descr(args.config, args.causal, getattr(args, "deterministic", False),
+                          args.shared_rows, args.per_head_rows)
     for _ in range(args.warmup):
         one()
     ts = [one() for _ in range(args.steps)]
@@ -255,7 +312,7 @@ def run_reference(args):
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _omp_threads(),
                              "kind": "oracle",
                              "sample": f"batch 0, head 0, {'last' if args.causal else 'first'} "
-                                       f"{sub.q.shape[2]} query rows "
+                                       f"{_rows_of(sub)} query rows "
                                        f"({pairs} kept pairs) per step"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -297,7 +354,8 @@ def run_ours(args):
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
 
-    p = workloads.make_config(args.config, args.batch, args.causal)
+    p = workloads.make_config(args.config, args.batch, args.causal, shared_rows=args.shared_rows,
+                              per_head_rows=args.per_head_rows, heads=args.heads)
     p.deterministic = args.deterministic
     pairs = _pairs(p)
     P = bsa.params_of_problem(p)
@@ -400,17 +458,29 @@ def run_ours(args):
         bwd_ktf = 10 * D * pairs / (bwd_kms * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         dominant = "bwd" if bwd_kms >= fwd_kms else "fwd"
-        achieved = bwd_ktf if dominant == "bwd" else fwd_ktf
-        traffic = (None if args.causal or args.deterministic
-                   else _traffic_from_profiles(args.config, dominant))
+        fwd_b, bwd_b = _alg_bytes(p)
+        dom_flops = (10 if dominant == "bwd" else 4) * D * pairs
+        dom_bytes = bwd_b if dominant == "bwd" else fwd_b
+        dom_ms = bwd_kms if dominant == "bwd" else fwd_kms
+        # below the ridge (FLOPs per algorithmic byte under peak FLOP/s over
+        # peak bytes/s) the kernel is held to the HBM roofline instead
+        hbm = dom_flops / dom_bytes < peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
+        achieved = (dom_bytes / (dom_ms * 1e-3) / 1e9 if hbm else
+                    (bwd_ktf if dominant == "bwd" else fwd_ktf))
+        rpeak = peaks["hbm_gbs"] if hbm else peak
+        variant = (args.causal or args.deterministic or args.shared_rows or args.batch is not None
+                   or args.heads is not None)
+        traffic = None if variant else _traffic_from_profiles(args.config, dominant)
         bwd_name = "k_bwd_tc+k_dq_tc" if args.deterministic else "k_bwd_tc"
         line = {
             "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if p.dtype == torch.bfloat16 else "f16", "data": "synthetic",
-            "config": {"workload": _descr(args.config, args.causal, args.deterministic)
-                       + ("" if args.batch is None else f" (batch overridden to {args.batch})"),
+            "config": {"workload": _descr(args.config, args.causal, args.deterministic,
+                                          args.shared_rows, args.per_head_rows)
+                       + ("" if args.batch is None else f" (batch overridden to {args.batch})")
+                       + ("" if args.heads is None else f" (heads overridden to {args.heads})"),
                        "kept_pairs_per_replica": pairs,
                        "parallelism": f"replicas x{world} (no exchange)",
                        "l2": "inputs larger than L2 (q/k/v/dout %d MiB each)"
@@ -419,12 +489,19 @@ def run_ours(args):
             "fwd_tflops": round(fwd_tf, 2), "bwd_tflops": round(bwd_tf, 2),
             "kernel_ms": {"k_fwd_tc": round(fwd_kms, 4), bwd_name: round(bwd_kms, 4)},
             "kernel_tflops": {"k_fwd_tc": round(fwd_ktf, 2), bwd_name: round(bwd_ktf, 2)},
+            "alg_bytes": {"fwd": fwd_b, "bwd": bwd_b},
+            "kernel_gbs": {"k_fwd_tc": round(fwd_b / (fwd_kms * 1e-3) / 1e9, 1),
+                           bwd_name: round(bwd_b / (bwd_kms * 1e-3) / 1e9, 1)},
             "pct_of_peak": round(100 * value / world / peak, 2),
-            "roofline": {"bound": "tensor", "kernel": bwd_name if dominant == "bwd" else "k_fwd_tc",
-                         "units": f"{10 if dominant == 'bwd' else 4}*D*kept_pairs FLOPs per launch",
-                         "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
-                         "frac": round(achieved / peak, 4), "peak_source": f"{which} bf16 burst",
-                         "frac_of_sustained": round(achieved / peaks.get("bf16_tflops_sustained", peak), 4),
+            "roofline": {"bound": "hbm" if hbm else "tensor",
+                         "kernel": bwd_name if dominant == "bwd" else "k_fwd_tc",
+                         "units": (f"{'backward' if dominant == 'bwd' else 'forward'} algorithmic bytes "
+                                   "per launch" if hbm else
+                                   f"{10 if dominant == 'bwd' else 4}*D*kept_pairs FLOPs per launch"),
+                         "achieved": round(achieved, 2), "peak": rpeak,
+                         "unit": "GB/s" if hbm else "TFLOP/s",
+                         "frac": round(achieved / rpeak, 4),
+                         "peak_source": f"{which} {'HBM copy' if hbm else 'bf16 burst'}",
                          "traffic": traffic},
             "e2e": {"value": round(job_tflops(world, step_flops, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -433,8 +510,12 @@ def run_ours(args):
             "status_flags": flags,
             "clocks": clk.summary(),
         }
+        if not hbm:
+            line["roofline"]["frac_of_sustained"] = round(
+                achieved / peaks.get("bf16_tflops_sustained", peak), 4)
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(args.config, causal=args.causal)
+            line["cpu_baseline"] = cpu_baseline(args.config, causal=args.causal,
+                                                shared_rows=args.shared_rows)
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -565,15 +646,25 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None,
                     help="smaller batch for C3/C4 (profiler captures only; not a bench line)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="fewer heads for C3/C4 (profiler captures only; not a bench line)")
     ap.add_argument("--causal", action="store_true",
                     help="C3 with the causal mask and its lower-triangular block index")
     ap.add_argument("--deterministic", action="store_true",
                     help="the deterministic backward (bitwise reproducible dq)")
     ap.add_argument("--fp8", action="store_true",
                     help="C3 with e4m3 q/k/v: the FP8 forward alone (one GPU)")
+    ap.add_argument("--shared-rows", action="store_true",
+                    help="C2/C5 with one index row per GQA group (packed forward tiles)")
+    ap.add_argument("--per-head-rows", action="store_true",
+                    help="with --shared-rows: the same rows copied to every query head")
     args = ap.parse_args()
     if args.causal and args.config != 3:
         ap.error("--causal applies to C3")
+    if args.shared_rows and args.config not in (2, 5):
+        ap.error("--shared-rows applies to C2 and C5")
+    if args.per_head_rows and not args.shared_rows:
+        ap.error("--per-head-rows needs --shared-rows")
     if args.impl == "reference":
         run_reference(args)
     elif args.fp8:

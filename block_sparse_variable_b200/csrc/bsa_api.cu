@@ -244,6 +244,13 @@ bsa_status prepare(const Args &a, Problem &p, Layout &L, bool &empty) {
   p.return_lse = want_lse ? 1 : 0;
   p.causal = P.mask_type == BSA_MASK_CAUSAL ? 1 : 0;
   p.deterministic = a.bwd && P.deterministic ? 1 : 0;
+  // GenericBlockSparseAttention, attribute table, isPackedGQA: the q heads of
+  // a group share the sparse pattern.  The forward then packs them into one
+  // tile whenever 128 / g rows per head is a whole number of 8-row swizzle
+  // atoms; the backward (kv-major) already streams K/V once per group.
+  const int64_t g = N1 / N2;
+  p.pack_g = (!a.bwd && Hidx == N2 && (g == 2 || g == 4 || g == 8 || g == 16)) ? int32_t(g) : 1;
+  p.fsub = int32_t(nsub * p.pack_g);
   p.fwd_slots = fwd_slots; p.bwd_slots = bwd_slots;
   p.fwd_slots_pad = fpad; p.bwd_slots_pad = bpad;
 

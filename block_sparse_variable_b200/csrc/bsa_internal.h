@@ -86,6 +86,13 @@ struct Problem {
   float *dsum;          // [rows_q][N1] rowsum(dOut o out)
   float *dq_acc;        // [rows_q][N1][D]; absent in the deterministic backward
   int64_t fwd_slots, bwd_slots, fwd_slots_pad, bwd_slots_pad;
+
+  // forward: query heads of a GQA group packed into one 128-row tile (the
+  // group shares its index row, Hidx == N2): each tile holds 128 / pack_g
+  // query rows of each of the pack_g heads, so every K/V chunk streamed in
+  // serves the whole group.  1 = one head per tile.
+  int32_t pack_g;
+  int32_t fsub;  // forward work items per query block: BQ * pack_g / 128
 };
 
 // ---- launchers (each returns the first launch error, cudaSuccess otherwise)

@@ -102,9 +102,16 @@ struct Layout {
   static_assert(kAlloc <= 232448, "shared memory budget");
 };
 
+template <bool kPack>
+__device__ __forceinline__ ItemView item_of(const Problem &p, int id) {
+  if constexpr (kPack) return item_view_packed(p, id);
+  else return item_view(p, id);
+}
+
 // kFp8: q, k, v in e4m3 (kind::f8f6f4 MMAs; P cast to e4m3 before P V);
-// BF16 then selects only the type of out
-template <int D, bool BF16, bool kCausal, bool kFp8>
+// BF16 then selects only the type of out.  kPack: packed-head items (the
+// query heads of a GQA group share the index row; p.pack_g heads per tile).
+template <int D, bool BF16, bool kCausal, bool kFp8, bool kPack>
 __global__ void __launch_bounds__(kTcThreads, 1)
     k_fwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
              const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v) {
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int armed_q = -1, armed[kStages] = {-1, -1, -1};
       bool ok = true;
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-        const ItemView v = item_view(p, p.fwd_items[it]);
+        const ItemView v = item_of<kPack>(p, p.fwd_items[it]);
         if (settle(p, v, Chunk{0, 0}).x >= v.ncnt) continue;  // no chunk: nothing to load
         if (is_k) {
           if (!(ok = wait_bar_lazy(bar(kBarQEmpty), (q_it & 1u) ^ 1u, abort, p.status))) break;
@@ -179,7 +186,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           armed_q = int(q_it & 1u);
           const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + v.t0 : v.t0;
           const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
-          tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, 0, v.h1, bb);
+          // packed heads: coordinates (0, row, first head, 0, batch)
+          if constexpr (kPack) tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, v.h1, 0, bb);
+          else tma_load_5d(sQ, &map_q, bar(kBarQFull), 0, tok, 0, v.h1, bb);
           ++q_it;
         }
         for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt; ch = next_chunk(p, v, ch)) {
@@ -200,9 +209,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             // the next item's Q tile into L2 as this item's last index entry
             // starts: its load waits for this item's last S, and a miss to
             // memory then would stall the pipeline
-            const ItemView w = item_view(p, p.fwd_items[it + gridDim.x]);
-            tma_prefetch_l2_5d(&map_q, 0, p.q_layout == BSA_LAYOUT_TND ? int(w.bi.q_tok0) + w.t0 : w.t0, 0,
-                               w.h1, p.q_layout == BSA_LAYOUT_TND ? 0 : w.b);
+            const ItemView w = item_of<kPack>(p, p.fwd_items[it + gridDim.x]);
+            const int wtok = p.q_layout == BSA_LAYOUT_TND ? int(w.bi.q_tok0) + w.t0 : w.t0;
+            const int wb = p.q_layout == BSA_LAYOUT_TND ? 0 : w.b;
+            if constexpr (kPack) tma_prefetch_l2_5d(&map_q, 0, wtok, w.h1, 0, wb);
+            else tma_prefetch_l2_5d(&map_q, 0, wtok, 0, w.h1, wb);
           }
           ++kv_it;
         }
@@ -246,7 +257,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t kv_it = 0, q_it = 0;
     bool ok = true;
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
-      const ItemView v = item_view(p, p.fwd_items[it]);
+      const ItemView v = item_of<kPack>(p, p.fwd_items[it]);
       const int n = count_chunks_warp(p, v, lane);
       if (n == 0) continue;
       if (is_s) {
@@ -302,7 +313,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp < kLoadWarp) {
     // --------------------------------------------- softmax warpgroups
     const int wg = warp >> 2;
-    const int r = tid & 127;  // query row = TMEM lane
+    const int r = tid & 127;  // tile row = TMEM lane
+    // the query row and head of tile row r (packed heads: 128/g rows per head)
+    const int rq = kPack ? r % (128 / p.pack_g) : r;
+    const int rh = kPack ? r / (128 / p.pack_g) : 0;
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     volatile uint32_t *flags = reinterpret_cast<volatile uint32_t *>(sbase + L::kFlags);
     float *xsum = reinterpret_cast<float *>(sbase + L::kXsum);
@@ -327,22 +341,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ItemView v;
         int coff;  // causal: the last kv token this row sees
         {
-          const ItemView full = item_view(p, p.fwd_items[it]);
+          const ItemView full = item_of<kPack>(p, p.fwd_items[it]);
           v.crow = full.crow;
           v.ncnt = full.ncnt;
           v.kvlen = full.kvlen;
           v.b = full.b;
           v.ksl = p.ksl;
           v.BKV = p.BKV;
-          coff = kCausal ? full.t0 + r + full.kvlen - full.bi.qlen : 0;
+          coff = kCausal ? full.t0 + rq + full.kvlen - full.bi.qlen : 0;
         }
-        for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok;
-             ch = next_chunk(p, v, ch), ++n, ++kv_it) {
+        for (Cursor ck = cur_begin(p, v); ck.x < v.ncnt && ok; cur_next(p, v, ck), ++n, ++kv_it) {
           const int b = int(kv_it % kSBufs);
           if (!(ok = wait_warp(bar(kBarSFull + b), (kv_it / kSBufs) & 1u, abort, p.status))) break;
           tc_fence_after();
           const uint32_t tS = tS0 + uint32_t(b) * 128u + lane_off;
-          const int u0c = v.u0(ch);
+          const int u0c = cur_u0(v, ck);
           const int valid_all = v.kvlen - u0c;             // kv columns of the chunk that exist
           // the chunk columns this row may see (causal: up to its own token)
           const int vis_all = kCausal ? min(valid_all, coff - u0c + 1) : valid_all;
@@ -478,9 +491,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (!ok) break;
       // ---- epilogue: out = O / sum of the groups' l; group w writes D/4 columns
-      const ItemView v = item_view(p, p.fwd_items[it]);
-      const bool live = r < v.rows;
-      T *orow = static_cast<T *>(p.out) + q_row(p.o_sb, p.o_sh, p.o_st, v.bi, v.b, v.h1, v.t0 + r);
+      const ItemView v = item_of<kPack>(p, p.fwd_items[it]);
+      const bool live = rq < v.rows;
+      T *orow = static_cast<T *>(p.out) + q_row(p.o_sb, p.o_sh, p.o_st, v.bi, v.b, v.h1 + rh, v.t0 + rq);
       if (n > 0) {
         const uint32_t t = kv_it - 1;  // the item's last P V; earlier ones precede it
         if (!(ok = wait_warp(bar(kBarPVDone + int(t & 1u)), (t / 2) & 1u, abort, p.status))) break;
@@ -496,7 +509,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
       for (int g2 = 0; g2 < kSoftmaxGroups; ++g2) Lsum += xs[g2 * 128 + r];
       if (wg == 0 && live && p.lse)
-        p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1, v.t0 + r)] =
+        p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, v.h1 + rh, v.t0 + rq)] =
             Lsum > 0.f ? (m + __log2f(Lsum)) * kLn2 : -INFINITY;
       const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
       if (n > 0) {
@@ -533,17 +546,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-template <int D, bool BF16, bool kCausal, bool kFp8 = false>
-cudaError_t launch_tc(const Problem &p, const FwdMaps &m, cudaStream_t s) {
+template <int D, bool BF16, bool kCausal, bool kFp8, bool kPack>
+cudaError_t launch_tc2(const Problem &p, const FwdMaps &m, cudaStream_t s) {
   // at least 120 KB so that exactly one CTA (the sole owner of all 512 TMEM
   // columns) is resident per SM
   const int smem = Layout<D, kFp8>::kAlloc > 120 * 1024 ? Layout<D, kFp8>::kAlloc : 120 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16, kCausal, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(k_fwd_tc<D, BF16, kCausal, kFp8, kPack>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int64_t grid = p.fwd_slots < num_sms() ? p.fwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_fwd_tc<D, BF16, kCausal, kFp8><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
+  k_fwd_tc<D, BF16, kCausal, kFp8, kPack><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
   return cudaGetLastError();
+}
+
+// packed-head items are a separate instantiation: the one-head kernel carries
+// none of their row mapping
+template <int D, bool BF16, bool kCausal, bool kFp8 = false>
+cudaError_t launch_tc(const Problem &p, const FwdMaps &m, cudaStream_t s) {
+  return p.pack_g > 1 ? launch_tc2<D, BF16, kCausal, kFp8, true>(p, m, s)
+                      : launch_tc2<D, BF16, kCausal, kFp8, false>(p, m, s);
 }
 
 }  // namespace

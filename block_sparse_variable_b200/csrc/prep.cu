@@ -110,8 +110,9 @@ __global__ void k_geometry(Problem p) {
   // the lengths need) select nothing: their rows get out 0 and lse -inf in
   // the forward, dq 0 in the deterministic backward (whose dq pass visits
   // work items only; the default backward converts every accumulator row).
+  // (BNSD indexes every batch with R = ceil(Sq/BQ) rows, checked on the host)
   const bool fwd = p.dq == nullptr;
-  if (s_sum_nq > p.R && (fwd || p.deterministic)) {
+  if (p.q_layout == BSA_LAYOUT_TND && s_sum_nq > p.R && (fwd || p.deterministic)) {
     const int CH = p.D / 8;  // 16-byte chunks of a 16-bit row
     for (int b = 0; b < p.B; ++b) {
       const BatchInfo bi = p.batch[b];
@@ -186,16 +187,28 @@ __global__ void k_compact(Problem p, int fwd_keys) {
   for (int w = n; w < p.W; ++w) dst[w] = kNoBlock;
   p.ncomp[r] = n;
   if (!fwd_keys) return;
-  const int h_lo = p.Hidx == p.N1 ? hi : hi * p.g;
-  const int h_hi = p.Hidx == p.N1 ? hi + 1 : h_lo + p.g;
   int made = 0;
-  for (int h1 = h_lo; h1 < h_hi; ++h1)
-    for (int qs = 0; qs < p.nsub; ++qs) {
-      const int64_t slot = (int64_t(h1) * p.Rg + gq) * p.nsub + qs;
-      const bool exists = b >= 0 && i * p.BQ + qs * kSlice < qlen;
+  if (p.pack_g > 1) {
+    // packed heads (Hidx == N2, hi = h2): slot (h2*Rg + gq)*fsub + s covers
+    // rows [s*R, s*R + R) of the query block for all g heads, R = 128/g
+    const int R = kSlice / p.pack_g;
+    for (int s = 0; s < p.fsub; ++s) {
+      const int64_t slot = (int64_t(hi) * p.Rg + gq) * p.fsub + s;
+      const bool exists = b >= 0 && i * p.BQ + s * R < qlen;
       p.keys[slot] = exists ? make_key(cost, slot) : kAbsentKey;
       made += exists;
     }
+  } else {
+    const int h_lo = p.Hidx == p.N1 ? hi : hi * p.g;
+    const int h_hi = p.Hidx == p.N1 ? hi + 1 : h_lo + p.g;
+    for (int h1 = h_lo; h1 < h_hi; ++h1)
+      for (int qs = 0; qs < p.nsub; ++qs) {
+        const int64_t slot = (int64_t(h1) * p.Rg + gq) * p.nsub + qs;
+        const bool exists = b >= 0 && i * p.BQ + qs * kSlice < qlen;
+        p.keys[slot] = exists ? make_key(cost, slot) : kAbsentKey;
+        made += exists;
+      }
+  }
   if (made) atomicAdd(p.status + kStFwdItems, uint32_t(made));
 }
 

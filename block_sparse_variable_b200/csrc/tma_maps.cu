@@ -38,10 +38,11 @@ int64_t esz(const Problem &p) { return p.dtype == BSA_F8E4M3 ? 1 : 2; }
 // {128/esz, 128, D*esz/128, 1, 1} lands as consecutive 128-row x 128-byte
 // boxes (16 KB each, 128-byte swizzle), i.e. a whole 128-row tile in one copy.
 cudaError_t encode(CUtensorMap *m, const Problem &p, const void *base, const cuuint64_t dims[5],
-                   const cuuint64_t strides[4]) {
+                   const cuuint64_t strides[4], const cuuint32_t *box_in = nullptr) {
   EncodeTiled fn = encoder();
   if (!fn) return cudaErrorNotSupported;
-  const cuuint32_t box[5] = {cuuint32_t(128 / esz(p)), 128, cuuint32_t(p.D * esz(p) / 128), 1, 1};
+  const cuuint32_t box_tile[5] = {cuuint32_t(128 / esz(p)), 128, cuuint32_t(p.D * esz(p) / 128), 1, 1};
+  const cuuint32_t *box = box_in ? box_in : box_tile;
   const cuuint32_t es[5] = {1, 1, 1, 1, 1};
   const CUtensorMapDataType dt = p.dtype == BSA_F8E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
                                  : p.dtype == BSA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
@@ -99,10 +100,27 @@ cudaError_t q_map(CUtensorMap *m, const Problem &p, const void *base, int64_t sb
   return encode(m, p, base, dims, strides);
 }
 
+// Packed-head query tiles: {128 B, token rows, q heads, groups, batch} with
+// box {128 B, 128/g, g, groups, 1}: the copy lands group by group, each group
+// head-major (g heads x 128/g rows of 128 bytes), i.e. one 128-row tile whose
+// row r is query row r % (128/g) of head r / (128/g).
+cudaError_t q_map_packed(CUtensorMap *m, const Problem &p) {
+  const int64_t e = esz(p);
+  const int64_t rows = p.q_layout == BSA_LAYOUT_TND ? p.Tq : p.Sq;
+  const int64_t nb = p.q_layout == BSA_LAYOUT_TND ? 1 : p.B;
+  const cuuint64_t dims[5] = {cuuint64_t(128 / e), cuuint64_t(rows), cuuint64_t(p.N1),
+                              cuuint64_t(p.D * e / 128), cuuint64_t(nb)};
+  const cuuint64_t strides[4] = {nz(p.q_st * e), nz(p.q_sh * e), 128,
+                                 nz(p.q_layout == BSA_LAYOUT_TND ? rows * p.q_st * e : p.q_sb * e)};
+  const cuuint32_t box[5] = {cuuint32_t(128 / e), cuuint32_t(128 / p.pack_g), cuuint32_t(p.pack_g),
+                             cuuint32_t(p.D * e / 128), 1};
+  return encode(m, p, p.q, dims, strides, box);
+}
+
 }  // namespace
 
 cudaError_t make_fwd_maps(const Problem &p, FwdMaps &m) {
-  cudaError_t e = q_map(&m.q, p, p.q, p.q_sb, p.q_sh, p.q_st);
+  cudaError_t e = p.pack_g > 1 ? q_map_packed(&m.q, p) : q_map(&m.q, p, p.q, p.q_sb, p.q_sh, p.q_st);
   if (e != cudaSuccess) return e;
   if ((e = kv_map(&m.k, p, p.k, p.k_sb, p.k_sh, p.k_st)) != cudaSuccess) return e;
   return kv_map(&m.v, p, p.v, p.v_sb, p.v_sh, p.v_st);

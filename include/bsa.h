@@ -274,7 +274,13 @@ const char *bsa_status_string(bsa_status status);
  *   inv_list   int32 batch-local query blocks per (index head, kv block)
  *   bwd_items  int32 backward item ids in execution order
  * Item ids: forward (h1*Rg + gq)*(BQ/128) + q_slice, gq the global query
- * block row; backward (h2*TK + gk)*(BKV/128) + kv_slice, gk the global kv
+ * block row, each item 128 query rows of head h1; but when the index is
+ * shared by the heads of a GQA group (Hidx == N2) with g = N1/N2 in
+ * {2, 4, 8, 16}, the forward packs the group (GenericBlockSparseAttention
+ * article, attribute isPackedGQA): (h2*Rg + gq)*(BQ*g/128) + slice, each item
+ * query rows [slice*128/g, (slice+1)*128/g) of the block for all g heads of
+ * kv head h2, so that every K/V chunk is streamed once for the group (the
+ * deterministic backward's q-major pass keeps one head per item); backward (h2*TK + gk)*(BKV/128) + kv_slice, gk the global kv
  * block (batch b's blocks after those of every earlier batch) and TK the
  * total kv blocks of this call (status word [5]). */
 typedef struct bsa_ws_region {

@@ -29,7 +29,12 @@ Definitions (the CUDA library must reproduce these exactly):
 * Forward work list: one item per (h1, gq, qsub) with qsub a 128-row slice
   of the q block holding at least one valid row; id = (h1*Rg + gq)*nsub +
   qsub, nsub = BQ/128; cost = number of (accepted block, 128-column slice)
-  pairs whose slice starts below kvlen_b.  Backward work list: one item per
+  pairs whose slice starts below kvlen_b.  When the g = N1/N2 query heads of
+  a group share their index row (Hidx == N2, GenericBlockSparseAttention
+  isPackedGQA) and g is 2, 4, 8 or 16, the forward packs them: one item per
+  (h2, gq, slice) with slice a run of R = 128/g rows of the q block holding
+  at least one valid row, id = (h2*Rg + gq)*(BQ/R) + slice, covering those
+  rows of all g heads; the cost is the same chunk count.  Backward work list: one item per
   (h2, gk, ksub) with the 128-row kv slice starting below kvlen_b; id =
   (h2*TK + gk)*ksubn + ksub; cost = sum over the group's q heads h1 and
   the listed q blocks i of the 128-row q slices holding a valid row.  Both
@@ -166,26 +171,42 @@ def inverted(p, geo: Geometry, comp, ncomp):
     return np.array(off, np.int32), np.array(lst, np.int32)
 
 
-def fwd_worklist(p, geo: Geometry, comp, ncomp):
-    """Item ids in execution order, and the cost of each slot id (-1: no item)."""
-    nsub, ksl = p.BQ // 128, p.BKV // 128
+def packed_heads(p) -> int:
+    """Query heads per forward item: g when the group shares its index row
+    and g is 2, 4, 8 or 16, else 1."""
     g = p.N1 // p.N2
+    return g if (p.Hidx == p.N2 and g in (2, 4, 8, 16)) else 1
+
+
+def fwd_worklist(p, geo: Geometry, comp, ncomp, packed=True):
+    """Item ids in execution order, and the cost of each slot id (-1: no item).
+    packed=False gives the one-head-per-item list (the deterministic
+    backward's q-major pass)."""
+    ksl = p.BKV // 128
+    g = p.N1 // p.N2
+    pg = packed_heads(p) if packed else 1
+    R = 128 // pg                      # query rows of one head per item
+    fsub = p.BQ // R                   # items per (head or group, q block)
+    nheads = p.N2 if pg > 1 else p.N1  # item heads: kv heads when packed
     Rg = geo.Rg
-    cost = np.full(p.N1 * Rg * nsub, -1, np.int64)
+    cost = np.full(nheads * Rg * fsub, -1, np.int64)
     for b in range(p.B):
         for i in range(geo.nq[b]):
             gq = geo.qoff[b] + i
             if gq >= Rg:
                 continue
-            for h1 in range(p.N1):
-                hi = h1 if p.Hidx == p.N1 else h1 // g
+            for hh in range(nheads):
+                if pg > 1:
+                    hi = hh
+                else:
+                    hi = hh if p.Hidx == p.N1 else hh // g
                 c = 0
                 for x in range(int(ncomp[hi, gq])):
                     j = int(comp[hi, gq, x])
                     c += sum(1 for s in range(ksl) if j * p.BKV + s * 128 < geo.kvlen[b])
-                for qs in range(nsub):
-                    if i * p.BQ + qs * 128 < geo.qlen[b]:
-                        cost[(h1 * Rg + gq) * nsub + qs] = c
+                for qs in range(fsub):
+                    if i * p.BQ + qs * R < geo.qlen[b]:
+                        cost[(hh * Rg + gq) * fsub + qs] = c
     ids = np.nonzero(cost >= 0)[0]
     order = np.lexsort((ids, -cost[ids]))
     return ids[order].astype(np.int32), cost
@@ -232,9 +253,11 @@ def build_all(p):
     comp, ncomp, f1 = compact(p, geo)
     off, lst = inverted(p, geo, comp, ncomp)
     fitems, fcost = fwd_worklist(p, geo, comp, ncomp)
+    fitems_1, _ = fwd_worklist(p, geo, comp, ncomp, packed=False)
     bitems, bcost = bwd_worklist(p, geo, off, lst)
     return {"geo": geo, "comp": comp, "ncomp": ncomp, "inv_off": off, "inv_list": lst,
-            "fwd_items": fitems, "fwd_cost": fcost, "bwd_items": bitems, "bwd_cost": bcost,
+            "fwd_items": fitems, "fwd_cost": fcost, "fwd_items_per_head": fitems_1,
+            "bwd_items": bitems, "bwd_cost": bcost,
             "flags": geo.flags | f1 | page_flags(p, geo)}
 
 

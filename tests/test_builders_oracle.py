@@ -51,6 +51,11 @@ RANDOM = [
          lens_kv=[1100, 333], Skv=1200, pattern=pat_density(0.6)),
     dict(layout_q="TND", layout_kv="PA_BBND", B=3, N1=2, N2=2, D=16, BQ=128, BKV=128,
          lens_q=[200, 300, 129], lens_kv=[500, 128, 1], page_size=128, pattern=pat_random_k),
+    # the group shares its index row, g = 4 and g = 8: packed forward items
+    dict(layout_q="TND", layout_kv="TND", B=3, N1=8, N2=2, Hidx=2, D=16, BQ=256, BKV=128,
+         lens_q=[300, 20, 530], lens_kv=[700, 90, 129], pattern=pat_density(0.5)),
+    dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=8, N2=1, Hidx=1, D=16, BQ=128, BKV=256,
+         Sq=300, lens_kv=[600, 257], Skv=600, pattern=pat_random_k),
 ]
 
 
@@ -103,5 +108,25 @@ def test_brute_force_token_mask(case):
             assert lst[off[li]:off[li + 1]].tolist() == sorted(inv.get((hi, gk), set()))
     want_f = [i for _, i in sorted((-c, i) for i, c in fcost.items())]
     want_b = [i for _, i in sorted((-c, i) for i, c in bcost.items())]
-    assert out["fwd_items"].tolist() == want_f
+    assert out["fwd_items_per_head"].tolist() == want_f
     assert out["bwd_items"].tolist() == want_b
+    # packed heads (the group shares its index row): one item per run of
+    # 128/g rows of a q block for all g heads, cost from the token mask of
+    # the group's first head at the run's first row
+    if p.Hidx == p.N2 and g in (2, 4, 8, 16):
+        R = 128 // g
+        fsub = p.BQ // R
+        pcost = {}
+        for b in range(p.B):
+            m = tr.token_mask(p, b).numpy()
+            for h2 in range(p.N2):
+                for i in range(geo.nq[b]):
+                    gq = geo.qoff[b] + i
+                    for s in range(fsub):
+                        t = i * p.BQ + s * R
+                        if t < geo.qlen[b]:
+                            pcost[(h2 * geo.Rg + gq) * fsub + s] = len(
+                                {u // 128 for u in np.nonzero(m[h2 * g, t])[0]})
+        assert out["fwd_items"].tolist() == [i for _, i in sorted((-c, i) for i, c in pcost.items())]
+    else:
+        assert out["fwd_items"].tolist() == want_f

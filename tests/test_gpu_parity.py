@@ -241,6 +241,63 @@ def test_corrupt_inputs_deterministic_backward(name):
     _check_deterministic(_corrupt(name))
 
 
+# Packed GQA tiles (GenericBlockSparseAttention, attribute isPackedGQA): the g
+# query heads of a group share their index row (Hidx == N2) and, for g in
+# {2, 4, 8, 16}, the forward packs 128/g rows of each head into one tile.
+# g = 3 shares the row but keeps one head per tile.
+PACKED = {
+    "packed_tnd_g4_d128": dict(layout_q="TND", layout_kv="TND", B=3, N1=16, N2=4, Hidx=4, D=128,
+                               lens_q=[300, 130, 517], lens_kv=[300, 700, 517],
+                               pattern=pat_fraction_diag(0.3)),
+    "packed_bnsd_g8": dict(layout_q="BNSD", layout_kv="BNSD", B=1, N1=8, N2=1, Hidx=1, D=64,
+                           Sq=300, BKV=256, pattern=pat_random_k),
+    "packed_bnsd_g16_bq256": dict(layout_q="BNSD", layout_kv="BNSD", B=2, N1=16, N2=1, Hidx=1,
+                                  D=64, Sq=200, BQ=256, pattern=pat_random_k),
+    "packed_paged_g4_fp16": dict(layout_q="TND", layout_kv="PA_BBND", B=3, N1=8, N2=2, Hidx=2,
+                                 D=128, lens_q=[300, 129, 64], lens_kv=[300, 129, 64],
+                                 page_size=128, extra_pages=2, dtype=torch.float16,
+                                 pattern=pat_topk(2)),
+    "packed_causal_g4": dict(layout_q="TND", layout_kv="TND", B=2, N1=8, N2=2, Hidx=2, D=64,
+                             lens_q=[300, 140], lens_kv=[500, 140], pattern=pat_dense, causal=True),
+    "packed_bq512_g2": dict(layout_q="TND", layout_kv="TND", B=2, N1=4, N2=2, Hidx=2, D=64,
+                            BQ=512, BKV=256, lens_q=[700, 300], lens_kv=[900, 300],
+                            pattern=pat_random_k),
+    "shared_rows_g3_unpacked": dict(layout_q="TND", layout_kv="TND", B=2, N1=6, N2=2, Hidx=2,
+                                    D=64, lens_q=[260, 140], lens_kv=[260, 300],
+                                    pattern=pat_random_k),
+}
+
+
+def _packed_problem(name):
+    return make_problem(seed_base=zlib.crc32(name.encode()) % 9973, name=name, **PACKED[name])
+
+
+@pytest.mark.parametrize("name", sorted(PACKED))
+def test_packed_gqa(name):
+    p = _packed_problem(name)
+    g = p.N1 // p.N2
+    assert builders.packed_heads(p) == (g if g in (2, 4, 8, 16) else 1)
+    _run_and_check(p)
+
+
+@pytest.mark.parametrize("name", ["packed_tnd_g4_d128", "packed_paged_g4_fp16", "packed_causal_g4"])
+def test_packed_gqa_equals_per_head_rows(name):
+    """The same problem with the group's row copied to every head (Hidx ==
+    N1, one head per tile) gives the same forward within rounding."""
+    p = _packed_problem(name)
+    g = p.N1 // p.N2
+    d = H.device_inputs(p)
+    out_p, lse_p, _, _ = H.gpu_fwd(p, d)
+    hdim = 1 if p.layout_q == "BNSD" else 0
+    p.index = p.index.view(torch.int16).repeat_interleave(g, dim=hdim).view(torch.uint16)
+    p.Hidx = p.N1
+    d = H.device_inputs(p)
+    out_h, lse_h, _, _ = H.gpu_fwd(p, d)
+    torch.cuda.synchronize()
+    H.check_close("out(packed vs per-head)", out_p, out_h.double())
+    H.check_lse(lse_p, lse_h)
+
+
 @pytest.mark.parametrize("name", sorted(SMALL))
 def test_small_cases(name):
     _run_and_check(_problem(name))
@@ -288,8 +345,9 @@ def _check_deterministic(p):
     st = H.region(ws_b, lay_b.status, torch.int32)
     B = builders.build_all(p)
     n_f = int(st[2])
-    assert n_f == len(B["fwd_items"])
-    assert np.array_equal(H.region(ws_b, lay_b.fwd_items, torch.int32, n_f), B["fwd_items"])
+    # the q-major pass takes one head per item, packed or not
+    assert n_f == len(B["fwd_items_per_head"])
+    assert np.array_equal(H.region(ws_b, lay_b.fwd_items, torch.int32, n_f), B["fwd_items_per_head"])
 
 
 @pytest.mark.parametrize("name", DETERMINISTIC)
@@ -476,6 +534,8 @@ FP8 = {
     "fp8_empty_rows": dict(layout_q="TND", layout_kv="TND", B=2, N1=2, N2=1, D=128,
                            lens_q=[384, 200], lens_kv=[256, 300], pattern=pat_random_k,
                            row_hook=_hook_empty),
+    "fp8_packed_g4": dict(layout_q="TND", layout_kv="TND", B=2, N1=8, N2=2, Hidx=2, D=128,
+                          lens_q=[300, 140], lens_kv=[400, 140], pattern=pat_random_k),
 }
 
 

@@ -264,18 +264,37 @@ def _lens(seed, B, lo, hi):
     return [int(x) for x in rng.integers(lo, hi + 1, size=B)]
 
 
-def make_config(c: int, batch: int | None = None, causal: bool = False, fp8: bool = False) -> Problem:
+def make_config(c: int, batch: int | None = None, causal: bool = False, fp8: bool = False,
+                shared_rows: bool = False, per_head_rows: bool = False,
+                heads: int | None = None) -> Problem:
     """C1..C5: the five workload shapes (see the module docstring for seeds).
 
-    `batch` overrides the batch of the BNSD shapes C3 and C4 (smaller cases
-    of the same kernels for profiler captures).  `causal` turns C3 into its
+    `batch` and `heads` (N1 = N2) override the batch and head count of the
+    BNSD shapes C3 and C4 (smaller cases of the same kernels for profiler
+    captures).  `causal` turns C3 into its
     causal variant: the causal mask with the lower-triangular block index;
     `fp8` gives C3 e4m3 q, k, v (bf16 out), the same N(0,1) draws rounded to
-    e4m3."""
+    e4m3.  `shared_rows` (C2, C5) draws one index row per GQA group instead
+    of one per query head (Hidx = N2, the GenericBlockSparseAttention
+    isPackedGQA pattern); `per_head_rows` then copies each group's row to
+    every query head of the group (Hidx = N1: the same selection, stated per
+    head)."""
+    if (shared_rows or per_head_rows) and c not in (2, 5):
+        raise ValueError("the shared-row variants are defined for C2 and C5")
+    if per_head_rows and not shared_rows:
+        raise ValueError("per_head_rows copies the rows of the shared-row variant")
+    if shared_rows:
+        q = make_config_shared(c)
+        if per_head_rows:
+            g = q.N1 // q.N2
+            q.index = q.index.view(torch.int16).repeat_interleave(g, dim=0).view(torch.uint16)
+            q.Hidx = q.N1
+            q.name += "-per-head-rows"
+        return q
     if fp8 and c != 3:
         raise ValueError("the FP8 variant is defined for C3 only")
-    if batch is not None and c not in (3, 4):
-        raise ValueError("batch override applies to C3 and C4 only")
+    if (batch is not None or heads is not None) and c not in (3, 4):
+        raise ValueError("batch / head overrides apply to C3 and C4 only")
     if causal and c != 3:
         raise ValueError("the causal variant is defined for C3 only")
     s = 1000 * c
@@ -290,12 +309,14 @@ def make_config(c: int, batch: int | None = None, causal: bool = False, fp8: boo
                             seed_base=s)
     if c == 3:
         return make_problem(name="C3-causal" if causal else "C3", layout_q="BNSD", layout_kv="BNSD",
-                            B=batch or 2, N1=32, N2=32, D=128, Sq=8192, BQ=128, BKV=512, W=16,
+                            B=batch or 2, N1=heads or 32, N2=heads or 32, D=128, Sq=8192, BQ=128,
+                            BKV=512, W=16,
                             pattern=pat_causal_blocks(128, 512) if causal else pat_dense,
                             seed_base=s, causal=causal,
                             dtype=torch.float8_e4m3fn if fp8 else torch.bfloat16)
     if c == 4:
-        return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=batch or 1, N1=24, N2=24, D=128,
+        return make_problem(name="C4", layout_q="BNSD", layout_kv="BNSD", B=batch or 1, N1=heads or 24,
+                            N2=heads or 24, D=128,
                             Sq=32768, BQ=128, BKV=128, W=256, pattern=pat_sink_diag_random(14),
                             seed_base=s)
     if c == 5:
@@ -304,6 +325,24 @@ def make_config(c: int, batch: int | None = None, causal: bool = False, fp8: boo
                             dtype=torch.float16, lens_q=lens, lens_kv=lens, BQ=128, BKV=128,
                             page_size=128, max_pages=32, W=8, pattern=pat_topk(8), seed_base=s)
     raise ValueError(f"unknown config C{c}")
+
+
+def make_config_shared(c: int) -> Problem:
+    """C2 / C5 with one index row per kv-head group (Hidx = N2), same seeds."""
+    s = 1000 * c
+    if c == 2:
+        lens = _lens(s + 6, 4, 256, 3072)
+        return make_problem(name="C2-shared-rows", layout_q="TND", layout_kv="TND", B=4, N1=16, N2=4,
+                            Hidx=4, D=128, lens_q=lens, lens_kv=lens, BQ=128, BKV=128,
+                            pattern=pat_fraction_diag(0.25), W=max(math.ceil(l / 128) for l in lens),
+                            seed_base=s)
+    if c == 5:
+        lens = _lens(s + 6, 8, 512, 4096)
+        return make_problem(name="C5-shared-rows", layout_q="TND", layout_kv="PA_BBND", B=8, N1=32,
+                            N2=8, Hidx=8, D=128, dtype=torch.float16, lens_q=lens, lens_kv=lens,
+                            BQ=128, BKV=128, page_size=128, max_pages=32, W=8, pattern=pat_topk(8),
+                            seed_base=s)
+    raise ValueError(f"no shared-row variant of C{c}")
 
 
 CONFIGS = {f"C{c}": c for c in range(1, 6)}
