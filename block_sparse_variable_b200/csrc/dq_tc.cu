@@ -302,12 +302,12 @@ __global__ void __launch_bounds__(kDThreads, 1)
       }
       const int coff = kCausal ? t + v.kvlen - v.bi.qlen : 0;  // last kv token this row sees
       int n = 0;
-      for (Chunk ch = settle(p, v, Chunk{0, 0}); ch.x < v.ncnt && ok; ch = next_chunk(p, v, ch), ++n, ++kv_it) {
+      for (Cursor ck = cur_begin(p, v); ck.x < v.ncnt && ok; cur_next(p, v, ck), ++n, ++kv_it) {
         const int b = int(kv_it & 1u), st = int(kv_it % kDStages);
         if (!(ok = wait_warp(bar(kDBarSFull + b), (kv_it >> 1) & 1u, abort, p.status))) break;
         if (!(ok = wait_warp(bar(kDBarDPFull), kv_it & 1u, abort, p.status))) break;
         tc_fence_after();
-        const int u0c = v.u0(ch);
+        const int u0c = cur_u0(v, ck);
         const int valid_all = v.kvlen - u0c;  // kv columns of the chunk that exist
         const int vis_all = kCausal ? min(valid_all, coff - u0c + 1) : valid_all;
         const int valid = vis_all - 64 * wg;  // of this group's columns
