@@ -81,7 +81,8 @@ struct BLayout {
   static constexpr int kBars = kStat + 2 * 256 * 4;
   static constexpr int kTmemPtr = kBars + kNumBars * 8;
   static constexpr int kAbort = kTmemPtr + 4;
-  static constexpr int kBytes = kAbort + 4;
+  static constexpr int kStepT0 = kAbort + 4;  // [2 slots] first query row of the step
+  static constexpr int kBytes = kStepT0 + 2 * 4;
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
@@ -154,6 +155,27 @@ __device__ __forceinline__ int b_t0(const Problem &p, const BItem &v, const BSte
   return b_qblock(p, v, c.hh, c.e, TK) * p.BQ + c.st * 128;
 }
 
+// The number of steps of an item (the walk of b_settle / b_next), by a whole
+// converged warp, once per item.  Without the dQ product (the deterministic
+// backward) the MMA issuer and the softmax warps count an item's steps this
+// way and take each step's first query row from the TMA warp (shared memory)
+// instead of walking the inverted index between two steps, which measured
+// faster there (and slower with the dQ product, whose kernel keeps the walk).
+__device__ __forceinline__ int b_count_steps_warp(const Problem &p, const BItem &v, int TK, int lane) {
+  int n = 0;
+  for (int hh = 0; hh < p.g; ++hh) {
+    const int64_t li = b_list(p, v, hh, TK);
+    const int off = p.inv_off[li], len = p.inv_off[li + 1] - off;
+    for (int e = lane; e < len; e += 32) {
+      const int rem = v.bi.qlen - p.inv_list[off + e] * p.BQ;  // query rows from the block start
+      n += rem > 0 ? min(p.nsub, (rem + 127) / 128) : 0;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) n += __shfl_xor_sync(0xffffffffu, n, o);
+  return n;
+}
+
 template <int D, bool BF16, bool kCausal, bool kDQ>
 __global__ void __launch_bounds__(kBThreads, 1)
     k_bwd_tc(const Problem p, const __grid_constant__ CUtensorMap map_q,
@@ -171,6 +193,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const uint32_t sK = base + L::kK, sV = base + L::kV, sQ = base + L::kQ, sDO = base + L::kDO;
   const uint32_t sDS = base + L::kDS;
   float *stat = reinterpret_cast<float *>(sbase + L::kStat);
+  int *step_t0 = reinterpret_cast<int *>(sbase + L::kStepT0);  // without dQ: per slot
   auto bar = [&](int i) { return base + L::kBars + 8u * uint32_t(i); };
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + L::kTmemPtr);
   volatile int *abort = reinterpret_cast<volatile int *>(sbase + L::kAbort);
@@ -289,6 +312,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
           st[lane + 32 * i] = l2r[i];
           st[128 + lane + 32 * i] = dsr[i];
         }
+        if constexpr (!kDQ)
+          if (lane == 0) step_t0[slot] = t0;
         __syncwarp();
         if (lane == 0) {
           if (kDQ && refill) reduce_slot(slot);
@@ -329,6 +354,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) continue;
+      const int n_steps = kDQ ? 0 : b_count_steps_warp(p, v, TK, lane);
       // the previous item's dK, dV must have been read out
       if (item_n > 0 && !(ok = wait_warp(bar(kBarAccFree), (item_n - 1) & 1u, abort, p.status))) break;
       ++item_n;
@@ -349,7 +375,9 @@ __global__ void __launch_bounds__(kBThreads, 1)
         __syncwarp();
       }
       bool first = true;
-      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
+      int s = 0;  // steps taken (without dQ: against the item's step count)
+      for (BStep c = kDQ ? b_settle(p, v, BStep{0, 0, 0}, TK) : BStep{0, 0, 0};
+           (kDQ ? c.hh < p.g : s < n_steps) && ok; c = kDQ ? b_next(p, v, c, TK) : c, ++s) {
         const int slot = int(sk & 1u);
         if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
         // R0 held the previous step's P and dS until its phase-2 MMAs were
@@ -424,10 +452,13 @@ __global__ void __launch_bounds__(kBThreads, 1)
       }
       const bool kv_ok = v.u0 + r < v.kvlen;
       int nsteps = 0;
-      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
+      const int n_steps = kDQ ? 0 : b_count_steps_warp(p, v, TK, lane);
+      for (BStep c = kDQ ? b_settle(p, v, BStep{0, 0, 0}, TK) : BStep{0, 0, 0};
+           (kDQ ? c.hh < p.g : nsteps < n_steps) && ok; c = kDQ ? b_next(p, v, c, TK) : c) {
         const int slot = int(sk & 1u);
-        const int t0 = b_t0(p, v, c, TK);
+        int t0 = kDQ ? b_t0(p, v, c, TK) : 0;
         if (!(ok = wait_warp(bar(kBarQD + slot), (sk >> 1) & 1u, abort, p.status))) break;
+        if constexpr (!kDQ) t0 = step_t0[slot];
         if (!(ok = wait_warp(bar(kBarS), sk & 1u, abort, p.status))) break;
         tc_fence_after();
         const float *lse2 = stat + slot * 256;
