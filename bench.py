@@ -184,7 +184,8 @@ def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = 
     """A bounded slice of the workload for the CPU oracle: batch 0, head 0,
     the first q_rows query rows against the full key range (causal: the
     last q_rows rows, which keeps every row's place relative to the end of
-    the kv sequence).  TND workloads: batch 0's first q_rows query rows of
+    the kv sequence); a BNSD slice of more rows than one head holds takes
+    whole heads 0..h-1 of batch 0.  TND workloads: batch 0's first q_rows query rows of
     head 0 against batch 0's kv rows of kv head 0 (gathered out of the pages
     for a paged cache: the same rows, stored contiguously)."""
     import workloads
@@ -207,17 +208,22 @@ def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = 
         sub.index = p.index[:1, :-(-q_rows // p.BQ)].contiguous()
         return sub
     S = p.q.shape[2]
+    # past one head's rows the slice takes whole heads of batch 0 (BNSD
+    # workloads here have one kv head per query head and one index row each)
+    h = 1
+    if q_rows > S and p.N1 == p.N2 == p.Hidx:
+        h = min(p.N1, q_rows // S)
     q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
-    sub = make_problem(B=1, N1=1, N2=1, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
+    sub = make_problem(B=1, N1=h, N2=h, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
                        BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale,
                        causal=causal, out_dtype=p.out_dtype)
     rows = slice(S - q_rows, S) if causal else slice(0, q_rows)
     blocks = slice(rows.start // p.BQ, rows.stop // p.BQ)
-    sub.q = p.q[:1, :1, rows].contiguous()
-    sub.k = p.k[:1, :1].contiguous()
-    sub.v = p.v[:1, :1].contiguous()
-    sub.dout = p.dout[:1, :1, rows].contiguous()
-    sub.index = p.index[:1, :1, blocks].contiguous()
+    sub.q = p.q[:1, :h, rows].contiguous()
+    sub.k = p.k[:1, :h].contiguous()
+    sub.v = p.v[:1, :h].contiguous()
+    sub.dout = p.dout[:1, :h, rows].contiguous()
+    sub.index = p.index[:1, :h, blocks].contiguous()
     sub.lens_q = [q_rows]
     return sub
 
@@ -255,14 +261,18 @@ def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False, shared_
     t = _oracle_step(sub)
     flops = 14 * sub.D * pairs
     return {"value": flops / t / 1e12, "unit": "TFLOP/s", "cores": _omp_threads(), "kind": "oracle",
-            "sample": f"fp64 oracle fwd+bwd on batch 0, head 0, {'last' if causal else 'first'} "
-                      f"{_rows_of(sub)} query rows "
+            "sample": f"fp64 oracle fwd+bwd on batch 0, {_heads_of(sub)}, "
+                      f"{'last' if causal else 'first'} {_rows_of(sub)} query rows "
                       f"x {sub.lens_kv[0]} keys of {DESCR[cfg].split(':')[0]} ({pairs} kept pairs, "
                       f"{t:.1f} s)"}
 
 
 def _rows_of(sub):
     return sub.q.shape[2] if sub.layout_q == "BNSD" else sub.q.shape[0]
+
+
+def _heads_of(sub):
+    return "head 0" if sub.N1 == 1 else f"heads 0..{sub.N1 - 1}"
 
 
 def _omp_threads():
@@ -311,7 +321,7 @@ def run_reference(args):
             "config": {"workload": workload, "sample": "see cpu_baseline"},
             "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": _omp_threads(),
                              "kind": "oracle",
-                             "sample": f"batch 0, head 0, {'last' if args.causal else 'first'} "
+                             "sample": f"batch 0, {_heads_of(sub)}, {'last' if args.causal else 'first'} "
                                        f"{_rows_of(sub)} query rows "
                                        f"({pairs} kept pairs) per step"},
             "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -613,14 +623,18 @@ def run_fp8(args):
         "gpu_launches": 5 * args.steps, "status_flags": flags, "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
-        sub = _oracle_subproblem(3, 8192, fp8=True)
         import oracle
-        t = time.perf_counter()
-        oracle.Oracle(sub).fwd()
-        t = time.perf_counter() - t
+
+        def fwd_time(sub):
+            t = time.perf_counter()
+            oracle.Oracle(sub).fwd()
+            return time.perf_counter() - t
+        t = fwd_time(_oracle_subproblem(3, 1024, fp8=True))
+        sub = _oracle_subproblem(3, int(1024 * max(1.0, 12.0 / max(t, 1e-3))), fp8=True)
+        t = fwd_time(sub)
         line["cpu_baseline"] = {"value": 4 * sub.D * _pairs(sub) / t / 1e12, "unit": "TFLOP/s",
                                 "cores": _omp_threads(), "kind": "oracle",
-                                "sample": f"fp64 oracle forward on batch 0, head 0, first "
+                                "sample": f"fp64 oracle forward on batch 0, {_heads_of(sub)}, first "
                                           f"{sub.q.shape[2]} query rows x {sub.k.shape[2]} keys ({t:.1f} s)"}
     print(json.dumps(line), flush=True)
 

@@ -60,3 +60,15 @@ def test_causal_blocks_pattern_is_exactly_the_reachable_blocks():
         last_visible = i * BQ + BQ - 1          # the block's last row sees up to its own token
         want = list(range(last_visible // BKV + 1))
         assert row == want, (i, row, want)
+
+
+def test_oracle_sample_takes_whole_heads_past_one_head():
+    """The CPU-baseline slice of C3 (dense index, S = 8192) grows by whole
+    heads once it asks for more rows than one head holds: each head keeps all
+    S x S pairs, and its tensors are the workload's own heads 0..h-1."""
+    sub = bench._oracle_subproblem(3, 3 * 8192 + 100)
+    assert sub.N1 == sub.N2 == 3 and sub.q.shape[1:3] == (3, 8192)
+    assert bench._pairs(sub) == 3 * 8192 * 8192
+    one = bench._oracle_subproblem(3, 1024)
+    assert one.N1 == 1 and bench._pairs(one) == 1024 * 8192
+    assert torch.equal(one.q[0, 0], sub.q[0, 0, :1024])
