@@ -24,24 +24,37 @@ __device__ __forceinline__ int64_t qstore_off(const Problem &p, int64_t sb, int6
   return r * st + int64_t(h) * sh;
 }
 
+// eight lanes per (query row, head): each reads 16 bytes of dOut and out per
+// pass (a warp covers four (row, head) pairs, 512 bytes of each tensor per
+// pass), then the eight partial dot products are summed by shuffles
 template <typename T>
 __global__ void k_bwd_pre(const Problem p) {
-  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= p.rows_q * p.N1) return;
-  const int64_t r = w / p.N1;
-  const int h = int(w % p.N1);
-  const T *dO = static_cast<const T *>(p.dout) + qstore_off(p, p.do_sb, p.do_sh, p.do_st, r, h);
-  const T *O = static_cast<const T *>(p.out) + qstore_off(p, p.o_sb, p.o_sh, p.o_st, r, h);
+  const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
+  const int sub = threadIdx.x & 7;
+  const bool live = w < p.rows_q * p.N1;
   float acc = 0.f;
-  for (int d = lane * 2; d < p.D; d += 64) {
-    const float2 a = Pack2<T>::unpack(*reinterpret_cast<const uint32_t *>(dO + d));
-    const float2 c = Pack2<T>::unpack(*reinterpret_cast<const uint32_t *>(O + d));
-    acc = fmaf(a.x, c.x, fmaf(a.y, c.y, acc));
+  int64_t r = 0;
+  int h = 0;
+  if (live) {
+    r = w / p.N1;
+    h = int(w % p.N1);
+    const T *dO = static_cast<const T *>(p.dout) + qstore_off(p, p.do_sb, p.do_sh, p.do_st, r, h);
+    const T *O = static_cast<const T *>(p.out) + qstore_off(p, p.o_sb, p.o_sh, p.o_st, r, h);
+    for (int d = sub * 8; d < p.D; d += 64) {
+      const uint4 a = *reinterpret_cast<const uint4 *>(dO + d);
+      const uint4 c = *reinterpret_cast<const uint4 *>(O + d);
+      const uint32_t av[4] = {a.x, a.y, a.z, a.w}, cv[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = Pack2<T>::unpack(av[e]);
+        const float2 y = Pack2<T>::unpack(cv[e]);
+        acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+      }
+    }
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-  if (lane == 0) p.dsum[r * p.N1 + h] = acc;
+  for (int o = 4; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (live && sub == 0) p.dsum[r * p.N1 + h] = acc;
 }
 
 // dq = dtype(scale * dQacc) for every q storage row
@@ -100,8 +113,8 @@ cudaError_t launch_bwd_pre(const Problem &p, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, size_t(p.rows_q) * p.N1 * p.D * sizeof(float), s);
     if (e != cudaSuccess) return e;
   }
-  const int64_t warps = p.rows_q * p.N1;
-  const unsigned grid = unsigned((warps * 32 + 255) / 256);
+  const int64_t pairs = p.rows_q * p.N1;  // eight lanes each
+  const unsigned grid = unsigned((pairs * 8 + 255) / 256);
   if (p.dtype == BSA_BF16) k_bwd_pre<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
   else k_bwd_pre<__half><<<grid, 256, 0, s>>>(p);
   return cudaGetLastError();

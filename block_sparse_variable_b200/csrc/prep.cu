@@ -9,7 +9,7 @@
 //     as CSR, plus the backward work of each (kv head, 128-row kv slice);
 //   * the load-balanced work lists: item ids sorted by cost descending then
 //     id ascending (longest first, ties head-major), by a per-CTA bitonic
-//     sort of 4096-key chunks followed by a merge by rank.
+//     sort of chunks of up to 4096 keys followed by a merge by rank.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -222,9 +222,13 @@ __device__ __forceinline__ bool row_has(const uint16_t *row, int n, int j) {
   return lo < n && int(row[lo]) == j;
 }
 
-// one thread per (index head, kv block); mode 0 counts, mode 1 fills
+// one warp per (index head, kv block) list: lane l tests query blocks l,
+// l + 32, ... of the kv block's batch (binary search in the compacted row);
+// mode 0 counts the blocks and their 128-row query slices, mode 1 writes the
+// ascending list (ballots give each hit its place)
 __global__ void k_inverse(Problem p, int mode) {
-  const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t idx = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
   if (idx >= int64_t(p.Hidx) * p.tk_max) return;
   const int hi = int(idx / p.tk_max);
   const int gk = int(idx % p.tk_max);
@@ -237,20 +241,30 @@ __global__ void k_inverse(Problem p, int mode) {
   if (b >= 0) {
     const BatchInfo bi = p.batch[b];
     const int j = gk - bi.koff;
-    for (int i = 0; i < bi.nq; ++i) {
+    for (int i0 = 0; i0 < bi.nq; i0 += 32) {
+      const int i = i0 + lane;
       const int64_t gq = int64_t(bi.qoff) + i;
-      if (gq >= p.Rg) break;
-      const int64_t rr = int64_t(hi) * p.Rg + gq;
-      if (row_has(p.comp + rr * p.W, p.ncomp[rr], j)) {
-        if (mode) p.inv_list[pos++] = i;
-        ++cnt;
+      bool hit = false;
+      if (i < bi.nq && gq < p.Rg) {
+        const int64_t rr = int64_t(hi) * p.Rg + gq;
+        hit = row_has(p.comp + rr * p.W, p.ncomp[rr], j);
+      }
+      const uint32_t m = __ballot_sync(0xffffffffu, hit);
+      if (hit) {
+        if (mode) p.inv_list[pos + __popc(m & ((1u << lane) - 1u))] = i;
         sub += min(p.nsub, (bi.qlen - i * p.BQ + kSlice - 1) / kSlice);
       }
+      pos += __popc(m);
+      cnt += __popc(m);
     }
   }
   if (!mode) {
-    p.inv_cnt[li] = cnt;
-    p.inv_sub[li] = sub;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sub += __shfl_xor_sync(0xffffffffu, sub, o);
+    if (lane == 0) {
+      p.inv_cnt[li] = cnt;
+      p.inv_sub[li] = sub;
+    }
   }
 }
 
@@ -322,43 +336,87 @@ __global__ void k_bwd_keys(Problem p) {
   if (exists) atomicAdd(p.status + kStBwdItems, 1u);
 }
 
-// bitonic sort of one kSortChunk-key chunk in shared memory (ascending)
-__global__ void __launch_bounds__(1024) k_sort_chunks(const uint64_t *keys, uint64_t *sorted,
-                                                      int64_t slots) {
+__device__ __forceinline__ void cmp_swap(uint64_t &a, uint64_t &c, bool up) {
+  if ((a > c) == up) { const uint64_t t = a; a = c; c = t; }
+}
+
+__device__ __forceinline__ uint64_t shfl_xor64(uint64_t x, int m) {
+  const uint32_t lo = __shfl_xor_sync(0xffffffffu, uint32_t(x), m);
+  const uint32_t hi = __shfl_xor_sync(0xffffffffu, uint32_t(x >> 32), m);
+  return (uint64_t(hi) << 32) | lo;
+}
+
+// bitonic sort (ascending) of one n-key chunk, n a power of two in
+// [128, kSortChunk], by n/4 threads; thread t holds keys 4t..4t+3 in
+// registers.  Stages whose partner distance j is 1 or 2 stay in the thread,
+// 4 <= j <= 64 cross lanes of one warp (shuffles), j >= 128 go through shared
+// memory, where consecutive such stages run in place.
+__global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *keys,
+                                                                uint64_t *sorted, int64_t slots,
+                                                                int n) {
   __shared__ uint64_t s[kSortChunk];
-  const int64_t base = int64_t(blockIdx.x) * kSortChunk;
-  for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x)
-    s[i] = base + i < slots ? keys[base + i] : kAbsentKey;
-  __syncthreads();
-  for (int k = 2; k <= kSortChunk; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x) {
-        const int ixj = i ^ j;
-        if (ixj > i) {
-          const uint64_t a = s[i], c = s[ixj];
-          const bool up = (i & k) == 0;
-          if ((a > c) == up) { s[i] = c; s[ixj] = a; }
+  const int t = threadIdx.x;
+  const int64_t base = int64_t(blockIdx.x) * n;
+  uint64_t v[4];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int64_t e = base + 4 * t + r;
+    v[r] = e < slots ? keys[e] : kAbsentKey;
+  }
+  for (int k = 2; k <= n; k <<= 1) {
+    int j = k >> 1;
+    if (j >= 128) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) s[4 * t + r] = v[r];
+      __syncthreads();
+      for (; j >= 128; j >>= 1) {
+        for (int q = t; q < (n >> 1); q += blockDim.x) {
+          const int i = ((q & ~(j - 1)) << 1) | (q & (j - 1));  // bit j of i clear
+          uint64_t a = s[i], c = s[i | j];
+          cmp_swap(a, c, (i & k) == 0);
+          s[i] = a;
+          s[i | j] = c;
         }
+        __syncthreads();
       }
+#pragma unroll
+      for (int r = 0; r < 4; ++r) v[r] = s[4 * t + r];
       __syncthreads();
     }
+    const bool up = ((4 * t) & k) == 0;  // the same for the thread's 4 keys once k >= 4
+    for (; j >= 4; j >>= 1) {
+      const bool keep_min = (((4 * t) & j) == 0) == up;
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const uint64_t o = shfl_xor64(v[r], j >> 2);
+        v[r] = keep_min ? (o < v[r] ? o : v[r]) : (o > v[r] ? o : v[r]);
+      }
+    }
+    if (j == 2) {
+      cmp_swap(v[0], v[2], up);
+      cmp_swap(v[1], v[3], up);
+    }
+    // j == 1 (for k == 2 the direction flips between the thread's two pairs)
+    cmp_swap(v[0], v[1], k == 2 ? true : up);
+    cmp_swap(v[2], v[3], k == 2 ? false : up);
   }
-  for (int i = threadIdx.x; i < kSortChunk; i += blockDim.x) sorted[base + i] = s[i];
+#pragma unroll
+  for (int r = 0; r < 4; ++r) sorted[base + 4 * t + r] = v[r];
 }
 
 // final position of every real key = its place in its chunk + the keys
 // below it in every other chunk (keys are unique: the id is in the low word)
-__global__ void k_rank(const uint64_t *sorted, int64_t nchunks, int32_t *items) {
+__global__ void k_rank(const uint64_t *sorted, int64_t nchunks, int n, int32_t *items) {
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (idx >= nchunks * kSortChunk) return;
+  if (idx >= nchunks * n) return;
   const uint64_t key = sorted[idx];
   if (key == kAbsentKey) return;
-  const int64_t c = idx / kSortChunk;
-  int64_t rank = idx - c * kSortChunk;
+  const int64_t c = idx / n;
+  int64_t rank = idx - c * n;
   for (int64_t o = 0; o < nchunks; ++o) {
     if (o == c) continue;
-    const uint64_t *a = sorted + o * kSortChunk;
-    int lo = 0, hi = kSortChunk;
+    const uint64_t *a = sorted + o * n;
+    int lo = 0, hi = n;
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       if (a[mid] < key) lo = mid + 1;
@@ -387,16 +445,20 @@ cudaError_t launch_prep_compact(const Problem &p, bool fwd_keys, cudaStream_t s)
 cudaError_t launch_sort_items(const Problem &p, int64_t slots_pad, int32_t *items, cudaStream_t s) {
   const bool fwd = items == p.fwd_items;
   const int64_t slots = fwd ? p.fwd_slots : p.bwd_slots;
-  const int64_t nchunks = slots_pad / kSortChunk;
-  if (nchunks == 0) return cudaGetLastError();
-  k_sort_chunks<<<unsigned(nchunks), 1024, 0, s>>>(p.keys, p.sorted, slots);
-  k_rank<<<unsigned((nchunks * kSortChunk + 255) / 256), 256, 0, s>>>(p.sorted, nchunks, items);
+  if (slots_pad == 0 || slots == 0) return cudaGetLastError();
+  // one chunk of the next power of two (at least 128) when the slots fit in
+  // one, else kSortChunk-key chunks (slots_pad is a multiple of kSortChunk)
+  int n = 128;
+  while (n < slots && n < kSortChunk) n <<= 1;
+  const int64_t nchunks = (slots + n - 1) / n;
+  k_sort_chunks<<<unsigned(nchunks), n / 4, 0, s>>>(p.keys, p.sorted, slots, n);
+  k_rank<<<unsigned((nchunks * n + 255) / 256), 256, 0, s>>>(p.sorted, nchunks, n, items);
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep_inverse(const Problem &p, cudaStream_t s) {
-  const int64_t n = int64_t(p.Hidx) * p.tk_max;
-  const unsigned grid = unsigned((n + 255) / 256);
+  const int64_t n = int64_t(p.Hidx) * p.tk_max;  // lists, one warp each
+  const unsigned grid = unsigned((n * 32 + 255) / 256);
   if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 0);
   k_scan_offsets<<<1, 1024, 0, s>>>(p);
   if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 1);
