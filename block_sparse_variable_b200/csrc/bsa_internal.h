@@ -24,6 +24,7 @@ enum : int {
   kStTK = 5,        // total kv blocks of this call
   kStNnz = 6,       // inverse-index entries
   kStSumNq = 7,     // query-block rows the lengths need
+  kStSubSum = 8,    // (2 words, uint64) sum of the inverse lists' 128-row query slices
   kStWords = 16
 };
 

@@ -65,8 +65,18 @@ enum : int {
   kBarAcc = 9,      // the item's dK, dV are final
   kBarAccFree = 10, // dK, dV read out (256 arrivals)
   kBarDrain = 11,
-  kNumBars = 12
+  kBarItemFull = 12,   // + ring slot: an item id is in the slot
+  kBarItemEmpty = 16,  // + ring slot: every consumer warp has read it (9 arrivals)
+  kNumBars = 20
 };
+
+// Work items are claimed at run time: a CTA's first item is its index, each
+// further one the next unclaimed entry of the list (a global counter), so
+// that the CTAs stay together on the list however unequal its items are.
+// The TMA warp claims them and passes the ids to the MMA issuer and the
+// softmax warps through a ring in shared memory.
+constexpr int kRing = 4;
+constexpr int kItemReaders = 9;  // the MMA warp and the eight softmax warps
 
 template <int D>
 struct BLayout {
@@ -82,7 +92,8 @@ struct BLayout {
   static constexpr int kTmemPtr = kBars + kNumBars * 8;
   static constexpr int kAbort = kTmemPtr + 4;
   static constexpr int kStepT0 = kAbort + 4;  // [2 slots] first query row of the step
-  static constexpr int kBytes = kStepT0 + 2 * 4;
+  static constexpr int kItems = kStepT0 + 2 * 4;  // [kRing] claimed item ids (-1: none left)
+  static constexpr int kBytes = kItems + kRing * 4;
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
@@ -194,6 +205,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const uint32_t sDS = base + L::kDS;
   float *stat = reinterpret_cast<float *>(sbase + L::kStat);
   int *step_t0 = reinterpret_cast<int *>(sbase + L::kStepT0);  // without dQ: per slot
+  volatile int *items_ring = reinterpret_cast<volatile int *>(sbase + L::kItems);
   auto bar = [&](int i) { return base + L::kBars + 8u * uint32_t(i); };
   volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(sbase + L::kTmemPtr);
   volatile int *abort = reinterpret_cast<volatile int *>(sbase + L::kAbort);
@@ -217,6 +229,10 @@ __global__ void __launch_bounds__(kBThreads, 1)
     mbar_init(bar(kBarAcc), 1);
     mbar_init(bar(kBarAccFree), 256);
     mbar_init(bar(kBarDrain), 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(bar(kBarItemFull + r), 1);
+      mbar_init(bar(kBarItemEmpty + r), kItemReaders);
+    }
     *abort = 0;
     fence_barrier_init();
   }
@@ -230,6 +246,18 @@ __global__ void __launch_bounds__(kBThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t tR0 = tmem, tR1 = tmem + 128u, tdV = tmem + 256u, tdK = tmem + 384u;
   const float kLog2e = 1.4426950408889634f;
+
+  // consumers: the next claimed item id from the ring (-1: none left, or abort)
+  uint32_t cseq = 0;
+  auto take_item = [&](bool &ok) -> int {
+    const int r = int(cseq % kRing);
+    if (!(ok = wait_warp(bar(kBarItemFull + r), (cseq / kRing) & 1u, abort, p.status))) return -1;
+    const int it = items_ring[r];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar(kBarItemEmpty + r));
+    ++cseq;
+    return it;
+  };
 
   if (warp == kBLoadWarp) {
     // ------------------------------------------------------ TMA producer
@@ -266,7 +294,29 @@ __global__ void __launch_bounds__(kBThreads, 1)
       __syncwarp();
       return true;
     };
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    // claim an item and hand its id (or -1 once the list is exhausted) to the
+    // consumers
+    uint32_t pseq = 0;
+    auto publish = [&](int it) -> int {
+      const int r = int(pseq % kRing);
+      if (pseq >= uint32_t(kRing) &&
+          !(ok = wait_warp_lazy(bar(kBarItemEmpty + r), (pseq / kRing - 1) & 1u, abort, p.status)))
+        return -1;
+      if (lane == 0) {
+        items_ring[r] = it;
+        mbar_arrive(bar(kBarItemFull + r));
+      }
+      __syncwarp();
+      ++pseq;
+      return it;
+    };
+    auto claim = [&]() -> int {
+      int nx = 0;
+      if (lane == 0) nx = int(gridDim.x) + int(atomicAdd(p.status + kStBwdNext, 1u));
+      nx = __shfl_sync(0xffffffffu, nx, 0);
+      return publish(nx < n_items ? nx : -1);
+    };
+    for (int it = publish(int(blockIdx.x) < n_items ? int(blockIdx.x) : -1); it >= 0 && ok; it = claim()) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) continue;
       if (!(ok = wait_warp_lazy(bar(kBarKVEmpty), (kv_it & 1u) ^ 1u, abort, p.status))) break;
@@ -351,7 +401,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     auto kstep = [](int kk) { return uint64_t((kk >> 2) * (L::kBox >> 4) + (kk & 3) * 2); };
     uint32_t kv_it = 0, sk = 0, item_n = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    for (int it = take_item(ok); it >= 0 && ok; it = take_item(ok)) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) continue;
       const int n_steps = kDQ ? 0 : b_count_steps_warp(p, v, TK, lane);
@@ -444,7 +494,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     const uint32_t lane_off = uint32_t((warp & 3) * 32) << 16;
     uint32_t sk = 0, item_n = 0;
     bool ok = true;
-    for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+    for (int it = take_item(ok); it >= 0 && ok; it = take_item(ok)) {
       const BItem v = b_item(p, p.bwd_items[it], TK);
       if (!v.steps_ok) {
         if (tid == 0) atomicOr(p.status + kStFlags, BSA_FLAG_BAD_PAGE);

@@ -268,17 +268,24 @@ __global__ void k_inverse(Problem p, int mode) {
   }
 }
 
-// single CTA exclusive scan of inv_cnt[0 .. Hidx*TK) into inv_off
+// single CTA exclusive scan of inv_cnt[0 .. Hidx*TK) into inv_off; also the
+// total of inv_sub (the backward work lists' grouping threshold)
 __global__ void k_scan_offsets(Problem p) {
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
+  __shared__ unsigned long long sub_total;
   const int64_t n = int64_t(p.Hidx) * p.status[kStTK];
-  if (threadIdx.x == 0) carry = 0;
+  if (threadIdx.x == 0) {
+    carry = 0;
+    sub_total = 0;
+  }
   __syncthreads();
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  unsigned long long my_sub = 0;
   for (int64_t base = 0; base < n; base += blockDim.x) {
     const int64_t i = base + threadIdx.x;
     const int32_t x = i < n ? p.inv_cnt[i] : 0;
+    if (i < n) my_sub += uint32_t(p.inv_sub[i]);
     int32_t s = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -303,10 +310,28 @@ __global__ void k_scan_offsets(Problem p) {
     if (threadIdx.x == blockDim.x - 1) carry = before + x;
     __syncthreads();
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_sub += __shfl_xor_sync(0xffffffffu, my_sub, o);
+  if (lane == 0) atomicAdd(&sub_total, my_sub);
+  __syncthreads();
   if (threadIdx.x == 0) {
     p.inv_off[n] = carry;
     p.status[kStNnz] = uint32_t(carry);
+    p.status[kStSubSum] = uint32_t(sub_total);
+    p.status[kStSubSum + 1] = uint32_t(sub_total >> 32);
   }
+}
+
+// Backward sort key.  Items whose cost exceeds 1/2048 of the list's total
+// (about 1/14 of a CTA's share on a 148-SM part) come first, longest first;
+// the rest follow kv head by kv head, longest first within a head, so that
+// the items in flight at any time share one kv head's Q, dOut and dQ rows
+// in L2.  (More than 1024 kv heads: longest first throughout.)
+__device__ __forceinline__ uint64_t bwd_key(int32_t cost, int h2, int64_t id, int64_t big) {
+  if (int64_t(cost) > big)
+    return (uint64_t(0x7FFFFFFFu - uint32_t(cost)) << 32) | uint64_t(uint32_t(id));
+  return (uint64_t(1) << 63) | (uint64_t(h2) << 53) |
+         (uint64_t(0x1FFFFFu - uint32_t(min(cost, 0x1FFFFF))) << 32) | uint64_t(uint32_t(id));
 }
 
 // one thread per backward slot (h2, gk, kv slice)
@@ -332,7 +357,13 @@ __global__ void k_bwd_keys(Problem p) {
       cost = p.g * p.inv_sub[int64_t(h2) * TK + gk];
     }
   }
-  p.keys[idx] = exists ? make_key(cost, idx) : kAbsentKey;
+  // the list's total cost, counting every kv block at full length: the sum of
+  // the inverse lists' query slices, times g when the group shares its lists,
+  // times the kv slices per block
+  const uint64_t sub = uint64_t(p.status[kStSubSum]) | (uint64_t(p.status[kStSubSum + 1]) << 32);
+  const int64_t total = int64_t(sub) * (p.Hidx == p.N1 ? 1 : p.g) * p.ksl;
+  const int64_t big = p.N2 <= 1024 ? total >> 11 : -1;
+  p.keys[idx] = exists ? bwd_key(cost, h2, idx, big) : kAbsentKey;
   if (exists) atomicAdd(p.status + kStBwdItems, 1u);
 }
 

@@ -262,8 +262,10 @@ const char *bsa_status_string(bsa_status status);
 /* Where the builders' results sit inside a workspace, so that callers (and
  * the tests) can inspect them after a call.  Offsets are bytes from the
  * workspace start; unused regions have bytes == 0.
- *   status     uint32[16]: [0] flags, [2] forward items, [4] backward items,
- *              [5] total kv blocks TK, [6] inverse-index entries
+ *   status     uint32[16]: [0] flags, [2] forward items, [3] backward items
+ *              claimed so far past the first one per CTA, [4] backward items,
+ *              [5] total kv blocks TK, [6] inverse-index entries, [8..9] the
+ *              inverse lists' 128-row query slices (uint64)
  *   batch      per batch 12 x int32: qlen, kvlen, nq, nk, qoff, koff,
  *              q_tok0 (2 words, int64), kv_tok0 (2 words, int64), kvst (kv
  *              rows stored for the batch), 1 spare
@@ -272,7 +274,9 @@ const char *bsa_status_string(bsa_status status);
  *   fwd_items  int32 forward item ids in execution order
  *   inv_off    int32 [Hidx*TK+1] CSR offsets of the KV-major inverse
  *   inv_list   int32 batch-local query blocks per (index head, kv block)
- *   bwd_items  int32 backward item ids in execution order
+ *   bwd_items  int32 backward item ids in the order the CTAs claim them:
+ *              the items above 1/2048 of the total cost first, longest
+ *              first, then kv head by kv head, longest first within a head
  * Item ids: forward (h1*Rg + gq)*(BQ/128) + q_slice, gq the global query
  * block row, each item 128 query rows of head h1; but when the index is
  * shared by the heads of a GQA group (Hidx == N2) with g = N1/N2 in

@@ -37,9 +37,12 @@ Definitions (the CUDA library must reproduce these exactly):
   rows of all g heads; the cost is the same chunk count.  Backward work list: one item per
   (h2, gk, ksub) with the 128-row kv slice starting below kvlen_b; id =
   (h2*TK + gk)*ksubn + ksub; cost = sum over the group's q heads h1 and
-  the listed q blocks i of the 128-row q slices holding a valid row.  Both
-  lists: cost descending, then id ascending (longest-processing-time first,
-  ties kept head-major).  Items of cost 0 stay: they write zeros.
+  the listed q blocks i of the 128-row q slices holding a valid row.  The
+  forward list: cost descending, then id ascending (longest-processing-time
+  first, ties kept head-major).  The backward list: the items whose cost
+  exceeds 1/2048 of the list's total first, cost descending; then the rest
+  kv head by kv head, cost descending within a head (bwd_worklist has the
+  exact rule).  Items of cost 0 stay: they write zeros.
 """
 from __future__ import annotations
 
@@ -231,8 +234,31 @@ def bwd_worklist(p, geo: Geometry, off, lst):
                     if j * p.BKV + ks * 128 < geo.kvlen[b]:
                         cost[(h2 * TK + gk) * ksl + ks] = c
     ids = np.nonzero(cost >= 0)[0]
-    order = np.lexsort((ids, -cost[ids]))
-    return ids[order].astype(np.int32), cost
+    # Order (the pages' metadata step balances the load but does not say
+    # how): the items above 1/2048 of the list's total cost first, longest
+    # first; then the rest kv head by kv head, longest first within a head
+    # (costs clamped at 2^21 - 1), ties by id.  The total counts every kv
+    # block at full length: the query slices of all inverse lists, times g
+    # when the group shares its lists, times the kv slices per block.
+    # (More than 1024 kv heads: longest first throughout.)
+    sub = 0
+    for hi in range(p.Hidx):
+        for b in range(p.B):
+            for j in range(geo.nk[b]):
+                li = hi * TK + geo.koff[b] + j
+                for i in lst[off[li]:off[li + 1]]:
+                    sub += sum(1 for qs in range(nsub) if int(i) * p.BQ + qs * 128 < geo.qlen[b])
+    total = sub * (1 if p.Hidx == p.N1 else g) * ksl
+    big = total >> 11 if p.N2 <= 1024 else -1
+
+    def key(i):
+        c = int(cost[i])
+        h2 = int(i) // (TK * ksl)
+        if c > big:
+            return (0, 0, -c, int(i))
+        return (1, h2, -min(c, (1 << 21) - 1), int(i))
+    order = sorted(ids.tolist(), key=key)
+    return np.asarray(order, dtype=np.int32), cost
 
 
 def page_flags(p, geo: Geometry) -> int:

@@ -59,6 +59,43 @@ RANDOM = [
 ]
 
 
+def _bwd_order(bcost, N2, per_head, ksl):
+    """The backward order from item costs alone: items above 1/2048 of the
+    total (every kv block counted at full length: slice 0's cost times the
+    slices per block) first by cost; then per kv head, by cost within it."""
+    total = sum(c * ksl for i, c in bcost.items() if i % ksl == 0)
+    big = total >> 11 if N2 <= 1024 else -1
+
+    def key(i):
+        c = bcost[i]
+        return (0, 0, -c, i) if c > big else (1, i // per_head, -min(c, (1 << 21) - 1), i)
+    return sorted(bcost, key=key)
+
+
+def test_bwd_order_groups_small_items_by_kv_head():
+    """With many kv heads the total is large enough that most items fall
+    below 1/2048 of it: those follow head by head, after the large ones;
+    costs counted here from the raw index rows (distinct in-range entries)."""
+    from workloads.gen import pat_sink_diag_random
+    p = make_problem(B=1, N1=48, N2=48, D=64, Sq=2048, BQ=128, BKV=128, W=8,
+                     pattern=pat_sink_diag_random(5), seed_base=321)
+    out = builders.build_all(p)
+    idx = p.index.view(torch.int16).numpy().view(np.uint16)
+    nq = nk = 2048 // 128
+    bcost = {}
+    for h in range(p.N2):
+        for j in range(nk):
+            bcost[h * nk + j] = sum(1 for i in range(nq)
+                                    if j in {int(e) for e in idx[0, h, i] if int(e) < nk})
+    want = _bwd_order(bcost, p.N2, nk, 1)
+    assert out["bwd_items"].tolist() == want
+    total = sum(bcost.values())
+    small = [i for i in want if bcost[i] <= total >> 11]
+    assert 0 < len(small) < len(want)            # both parts present
+    heads = [i // nk for i in small]
+    assert heads == sorted(heads)                # the small items head by head
+
+
 @pytest.mark.parametrize("case", range(len(RANDOM)))
 def test_brute_force_token_mask(case):
     """Compaction == sorted distinct entries; inverse == transpose of the
@@ -107,9 +144,8 @@ def test_brute_force_token_mask(case):
             li = hi * geo.TK + gk
             assert lst[off[li]:off[li + 1]].tolist() == sorted(inv.get((hi, gk), set()))
     want_f = [i for _, i in sorted((-c, i) for i, c in fcost.items())]
-    want_b = [i for _, i in sorted((-c, i) for i, c in bcost.items())]
     assert out["fwd_items_per_head"].tolist() == want_f
-    assert out["bwd_items"].tolist() == want_b
+    assert out["bwd_items"].tolist() == _bwd_order(bcost, p.N2, geo.TK * ksl, ksl)
     # packed heads (the group shares its index row): one item per run of
     # 128/g rows of a q block for all g heads, cost from the token mask of
     # the group's first head at the run's first row
