@@ -322,8 +322,8 @@ __global__ void k_scan_offsets(Problem p) {
   }
 }
 
-// Backward sort key.  Items whose cost exceeds 1/2048 of the list's total
-// (about 1/14 of a CTA's share on a 148-SM part) come first, longest first;
+// Backward sort key.  Items whose cost exceeds 1/512 of the list's total
+// (about 0.3 of a CTA's share on a 148-SM part) come first, longest first;
 // the rest follow kv head by kv head, longest first within a head, so that
 // the items in flight at any time share one kv head's Q, dOut and dQ rows
 // in L2.  (More than 1024 kv heads: longest first throughout.)
@@ -362,7 +362,7 @@ __global__ void k_bwd_keys(Problem p) {
   // times the kv slices per block
   const uint64_t sub = uint64_t(p.status[kStSubSum]) | (uint64_t(p.status[kStSubSum + 1]) << 32);
   const int64_t total = int64_t(sub) * (p.Hidx == p.N1 ? 1 : p.g) * p.ksl;
-  const int64_t big = p.N2 <= 1024 ? total >> 11 : -1;
+  const int64_t big = p.N2 <= 1024 ? total >> 9 : -1;
   p.keys[idx] = exists ? bwd_key(cost, h2, idx, big) : kAbsentKey;
   if (exists) atomicAdd(p.status + kStBwdItems, 1u);
 }

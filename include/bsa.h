@@ -275,7 +275,7 @@ const char *bsa_status_string(bsa_status status);
  *   inv_off    int32 [Hidx*TK+1] CSR offsets of the KV-major inverse
  *   inv_list   int32 batch-local query blocks per (index head, kv block)
  *   bwd_items  int32 backward item ids in the order the CTAs claim them:
- *              the items above 1/2048 of the total cost first, longest
+ *              the items above 1/512 of the total cost first, longest
  *              first, then kv head by kv head, longest first within a head
  * Item ids: forward (h1*Rg + gq)*(BQ/128) + q_slice, gq the global query
  * block row, each item 128 query rows of head h1; but when the index is

@@ -40,7 +40,7 @@ Definitions (the CUDA library must reproduce these exactly):
   the listed q blocks i of the 128-row q slices holding a valid row.  The
   forward list: cost descending, then id ascending (longest-processing-time
   first, ties kept head-major).  The backward list: the items whose cost
-  exceeds 1/2048 of the list's total first, cost descending; then the rest
+  exceeds 1/512 of the list's total first, cost descending; then the rest
   kv head by kv head, cost descending within a head (bwd_worklist has the
   exact rule).  Items of cost 0 stay: they write zeros.
 """
@@ -235,7 +235,7 @@ def bwd_worklist(p, geo: Geometry, off, lst):
                         cost[(h2 * TK + gk) * ksl + ks] = c
     ids = np.nonzero(cost >= 0)[0]
     # Order (the pages' metadata step balances the load but does not say
-    # how): the items above 1/2048 of the list's total cost first, longest
+    # how): the items above 1/512 of the list's total cost first, longest
     # first; then the rest kv head by kv head, longest first within a head
     # (costs clamped at 2^21 - 1), ties by id.  The total counts every kv
     # block at full length: the query slices of all inverse lists, times g
@@ -249,7 +249,7 @@ def bwd_worklist(p, geo: Geometry, off, lst):
                 for i in lst[off[li]:off[li + 1]]:
                     sub += sum(1 for qs in range(nsub) if int(i) * p.BQ + qs * 128 < geo.qlen[b])
     total = sub * (1 if p.Hidx == p.N1 else g) * ksl
-    big = total >> 11 if p.N2 <= 1024 else -1
+    big = total >> 9 if p.N2 <= 1024 else -1
 
     def key(i):
         c = int(cost[i])

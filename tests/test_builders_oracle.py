@@ -60,11 +60,11 @@ RANDOM = [
 
 
 def _bwd_order(bcost, N2, per_head, ksl):
-    """The backward order from item costs alone: items above 1/2048 of the
+    """The backward order from item costs alone: items above 1/512 of the
     total (every kv block counted at full length: slice 0's cost times the
     slices per block) first by cost; then per kv head, by cost within it."""
     total = sum(c * ksl for i, c in bcost.items() if i % ksl == 0)
-    big = total >> 11 if N2 <= 1024 else -1
+    big = total >> 9 if N2 <= 1024 else -1
 
     def key(i):
         c = bcost[i]
@@ -74,7 +74,7 @@ def _bwd_order(bcost, N2, per_head, ksl):
 
 def test_bwd_order_groups_small_items_by_kv_head():
     """With many kv heads the total is large enough that most items fall
-    below 1/2048 of it: those follow head by head, after the large ones;
+    below 1/512 of it: those follow head by head, after the large ones;
     costs counted here from the raw index rows (distinct in-range entries)."""
     from workloads.gen import pat_sink_diag_random
     p = make_problem(B=1, N1=48, N2=48, D=64, Sq=2048, BQ=128, BKV=128, W=8,
@@ -90,7 +90,7 @@ def test_bwd_order_groups_small_items_by_kv_head():
     want = _bwd_order(bcost, p.N2, nk, 1)
     assert out["bwd_items"].tolist() == want
     total = sum(bcost.values())
-    small = [i for i in want if bcost[i] <= total >> 11]
+    small = [i for i in want if bcost[i] <= total >> 9]
     assert 0 < len(small) < len(want)            # both parts present
     heads = [i // nk for i in small]
     assert heads == sorted(heads)                # the small items head by head
