@@ -212,7 +212,7 @@ def _oracle_subproblem(cfg: int, q_rows: int, causal: bool = False, fp8: bool = 
     # workloads here have one kv head per query head and one index row each)
     h = 1
     if q_rows > S and p.N1 == p.N2 == p.Hidx:
-        h = min(p.N1, q_rows // S)
+        h = min(p.N1, (q_rows + S // 2) // S)  # the nearest whole number of heads
     q_rows = max(p.BQ, min(S, (q_rows // p.BQ) * p.BQ))
     sub = make_problem(B=1, N1=h, N2=h, D=p.D, Sq=q_rows, Skv=p.k.shape[2], lens_kv=[p.lens_kv[0]],
                        BQ=p.BQ, BKV=p.BKV, W=p.W, pattern=pat_dense, dtype=p.dtype, scale=p.scale,
