@@ -39,6 +39,7 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
+#include "f32x2.cuh"
 #include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -337,7 +338,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         const int t0 = b_t0(p, v, c, TK);
         // lse (log2 units) and Dsum of the step's 128 query rows, fetched
         // before waiting for the slot; rows past qlen get lse = +inf (so
-        // P = 0) and Dsum = 0
+        // P = 0) and Dsum = 0.  Both are staged negated, as the addends of
+        // the softmax warps' paired fp32 operations.
         float l2r[4], dsr[4];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -359,8 +361,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
         float *st = stat + slot * 256;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          st[lane + 32 * i] = l2r[i];
-          st[128 + lane + 32 * i] = dsr[i];
+          st[lane + 32 * i] = -l2r[i];
+          st[128 + lane + 32 * i] = -dsr[i];
         }
         if constexpr (!kDQ)
           if (lane == 0) step_t0[slot] = t0;
@@ -535,14 +537,20 @@ __global__ void __launch_bounds__(kBThreads, 1)
 #pragma unroll
             for (int c2 = 0; c2 < 16; c2 += 2) {
               const int q = int(c0) + 16 * k + c2;
-              float p0 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2]), p.scale_log2, -lse2[q])) : 0.f;
-              float p1 = kv_ok ? ex2(fmaf(__uint_as_float(bs[c2 + 1]), p.scale_log2, -lse2[q + 1])) : 0.f;
+              // lse2 and dsum hold -lse*log2(e) and -Dsum (pairs of columns)
+              const float2 a2 = fma2(make_float2(__uint_as_float(bs[c2]), __uint_as_float(bs[c2 + 1])),
+                                     make_float2(p.scale_log2, p.scale_log2),
+                                     *reinterpret_cast<const float2 *>(lse2 + q));
+              float p0 = kv_ok ? ex2(a2.x) : 0.f;
+              float p1 = kv_ok ? ex2(a2.y) : 0.f;
               if constexpr (decltype(masked)::value) {
                 p0 = q >= qmin ? p0 : 0.f;
                 p1 = q + 1 >= qmin ? p1 : 0.f;
               }
-              const float s0 = p0 * (__uint_as_float(bd[c2]) - dsum[q]);
-              const float s1 = p1 * (__uint_as_float(bd[c2 + 1]) - dsum[q + 1]);
+              const float2 t2 = add2(make_float2(__uint_as_float(bd[c2]), __uint_as_float(bd[c2 + 1])),
+                                     *reinterpret_cast<const float2 *>(dsum + q));
+              const float2 s2 = mul2(make_float2(p0, p1), t2);
+              const float s0 = s2.x, s1 = s2.y;
               pp[8 * k + (c2 >> 1)] = Pack2<T>::pack(p0, p1);
               dd[8 * k + (c2 >> 1)] = Pack2<T>::pack(s0, s1);
             }

@@ -38,6 +38,7 @@
 #include "coalesce.cuh"
 #include "bsa_internal.h"
 #include "fwd_walk.cuh"
+#include "f32x2.cuh"
 #include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -331,10 +332,14 @@ __global__ void __launch_bounds__(kDThreads, 1)
 #pragma unroll
             for (int c2 = 0; c2 < 16; c2 += 2) {
               const int c = 16 * k + c2;
-              float s0 = ex2(fmaf(__uint_as_float(bs[c2]), p.scale_log2, -lse2)) *
-                         (__uint_as_float(bd[c2]) - dsum);
-              float s1 = ex2(fmaf(__uint_as_float(bs[c2 + 1]), p.scale_log2, -lse2)) *
-                         (__uint_as_float(bd[c2 + 1]) - dsum);
+              // the pair's P and dS by paired fp32 operations (the same bits as
+              // the scalar forms)
+              const float2 a2 = fma2(make_float2(__uint_as_float(bs[c2]), __uint_as_float(bs[c2 + 1])),
+                                     make_float2(p.scale_log2, p.scale_log2), make_float2(-lse2, -lse2));
+              const float2 t2 = add2(make_float2(__uint_as_float(bd[c2]), __uint_as_float(bd[c2 + 1])),
+                                     make_float2(-dsum, -dsum));
+              const float2 s2 = mul2(make_float2(ex2(a2.x), ex2(a2.y)), t2);
+              float s0 = s2.x, s1 = s2.y;
               if constexpr (decltype(masked)::value) {
                 // columns past the used length or (causal) past the row's
                 // last visible token: exactly 0, whatever S and dP hold there
