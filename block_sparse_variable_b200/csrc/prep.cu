@@ -394,6 +394,21 @@ __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *
     const int64_t e = base + 4 * t + r;
     v[r] = e < slots ? keys[e] : kAbsentKey;
   }
+  // a chunk already in order (equal costs: the keys ascend with the id)
+  // needs no network
+  {
+    const uint64_t next = __shfl_down_sync(0xffffffffu, v[0], 1);
+    bool in_order = v[0] <= v[1] && v[1] <= v[2] && v[2] <= v[3] &&
+                    ((t & 31) == 31 || v[3] <= next);
+    if ((t & 31) == 0) s[t >> 5] = v[0];  // each warp's first key, for the warp before
+    __syncthreads();
+    if ((t & 31) == 31 && t + 1 < int(blockDim.x)) in_order = in_order && v[3] <= s[(t >> 5) + 1];
+    if (__syncthreads_and(in_order)) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) sorted[base + 4 * t + r] = v[r];
+      return;
+    }
+  }
   for (int k = 2; k <= n; k <<= 1) {
     int j = k >> 1;
     if (j >= 128) {
