@@ -86,10 +86,11 @@ def _load():
     lib.bsa_selftest_exp2.argtypes = [vp, vp, vp, ctypes.c_int64, vp]
     lib.bsa_selftest_e4m3.argtypes = [vp, vp, ctypes.c_int64, vp]
     lib.bsa_selftest_wait_timeout.argtypes = [vp, vp]
+    lib.bsa_selftest_f32x2.argtypes = [vp, vp, vp, vp, vp, ctypes.c_int64, vp]
     for f in ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_fwd_workspace_layout",
               "bsa_bwd_get_workspace", "bsa_bwd", "bsa_bwd_workspace_layout", "bsa_read_status",
               "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout",
-              "bsa_selftest_e4m3"):
+              "bsa_selftest_e4m3", "bsa_selftest_f32x2"):
         getattr(lib, f).restype = ctypes.c_int
     return lib
 
@@ -100,7 +101,7 @@ EXPORTED = ("bsa_fwd_get_workspace", "bsa_fwd", "bsa_bwd_get_workspace", "bsa_bw
             "bsa_read_status", "bsa_status_string", "bsa_fwd_workspace_layout",
             "bsa_bwd_workspace_layout", "bsa_abi_version", "bsa_fwd_static_workspace",
             "bsa_set_main_kernel_events", "bsa_selftest_exp2", "bsa_selftest_wait_timeout",
-            "bsa_selftest_e4m3")
+            "bsa_selftest_e4m3", "bsa_selftest_f32x2")
 
 
 def lib():
@@ -341,6 +342,20 @@ def bsa_selftest_e4m3(x: torch.Tensor, stream=None) -> torch.Tensor:
     _check(_lib.bsa_selftest_e4m3(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()),
                                   x.numel(), ctypes.c_void_p(_stream(stream))), "bsa_selftest_e4m3")
     return y.view(torch.uint8)
+
+
+def bsa_selftest_f32x2(a: torch.Tensor, b: torch.Tensor, c: torch.Tensor, stream=None):
+    """(paired, scalar) results of fma(a,b,c), a+b and a*b for CUDA float32
+    tensors of one even numel; each a float32 tensor [3, numel]."""
+    a, b, c = (t.contiguous() for t in (a, b, c))
+    n = a.numel()
+    pair = torch.empty(3, n, dtype=torch.float32, device=a.device)
+    scal = torch.empty_like(pair)
+    _check(_lib.bsa_selftest_f32x2(ctypes.c_void_p(a.data_ptr()), ctypes.c_void_p(b.data_ptr()),
+                                   ctypes.c_void_p(c.data_ptr()), ctypes.c_void_p(pair.data_ptr()),
+                                   ctypes.c_void_p(scal.data_ptr()), n,
+                                   ctypes.c_void_p(_stream(stream))), "bsa_selftest_f32x2")
+    return pair, scal
 
 
 def bsa_selftest_wait_timeout(flags: torch.Tensor, stream=None):

@@ -11,6 +11,7 @@
 
 #include "addr.cuh"
 #include "bsa_internal.h"
+#include "launch.cuh"
 #include "pack16.cuh"
 
 namespace bsa {
@@ -29,6 +30,8 @@ __device__ __forceinline__ int64_t qstore_off(const Problem &p, int64_t sb, int6
 // pass), then the eight partial dot products are summed by shuffles
 template <typename T>
 __global__ void k_bwd_pre(const Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t w = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 3;
   const int sub = threadIdx.x & 7;
   const bool live = w < p.rows_q * p.N1;
@@ -60,6 +63,8 @@ __global__ void k_bwd_pre(const Problem p) {
 // dq = dtype(scale * dQacc) for every q storage row
 template <typename T>
 __global__ void k_dq_convert(const Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t n8 = p.rows_q * p.N1 * (p.D / 8);
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= n8) return;
@@ -82,6 +87,8 @@ __global__ void k_dq_convert(const Problem p) {
 // [round_up(kvlen, 128), kvst) -- stored rows past the used length
 template <typename T>
 __global__ void k_kv_zero_tail(const Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   const int b = blockIdx.y;
   const BatchInfo bi = p.batch[b];
   const int lo = ((bi.kvlen + kSlice - 1) / kSlice) * kSlice;
@@ -115,8 +122,9 @@ cudaError_t launch_bwd_pre(const Problem &p, cudaStream_t s) {
   }
   const int64_t pairs = p.rows_q * p.N1;  // eight lanes each
   const unsigned grid = unsigned((pairs * 8 + 255) / 256);
-  if (p.dtype == BSA_BF16) k_bwd_pre<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
-  else k_bwd_pre<__half><<<grid, 256, 0, s>>>(p);
+  cudaError_t e = p.dtype == BSA_BF16 ? launch_dep(k_bwd_pre<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, p)
+                                      : launch_dep(k_bwd_pre<__half>, dim3(grid), dim3(256), 0, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
@@ -124,13 +132,17 @@ cudaError_t launch_bwd_post(const Problem &p, cudaStream_t s) {
   const int64_t n8 = p.rows_q * p.N1 * (p.D / 8);
   const unsigned grid = unsigned((n8 + 255) / 256);
   const dim3 zgrid(64, unsigned(p.B));
+  cudaError_t e = cudaSuccess;
   if (p.dtype == BSA_BF16) {
-    if (p.dq_acc) k_dq_convert<__nv_bfloat16><<<grid, 256, 0, s>>>(p);
-    k_kv_zero_tail<__nv_bfloat16><<<zgrid, 256, 0, s>>>(p);
+    if (p.dq_acc && (e = launch_dep(k_dq_convert<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, p)) != cudaSuccess)
+      return e;
+    e = launch_dep(k_kv_zero_tail<__nv_bfloat16>, zgrid, dim3(256), 0, s, p);
   } else {
-    if (p.dq_acc) k_dq_convert<__half><<<grid, 256, 0, s>>>(p);
-    k_kv_zero_tail<__half><<<zgrid, 256, 0, s>>>(p);
+    if (p.dq_acc && (e = launch_dep(k_dq_convert<__half>, dim3(grid), dim3(256), 0, s, p)) != cudaSuccess)
+      return e;
+    e = launch_dep(k_kv_zero_tail<__half>, zgrid, dim3(256), 0, s, p);
   }
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

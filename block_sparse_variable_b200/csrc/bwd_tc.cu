@@ -40,6 +40,7 @@
 #include "addr.cuh"
 #include "bsa_internal.h"
 #include "f32x2.cuh"
+#include "launch.cuh"
 #include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -196,6 +197,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
   using L = BLayout<D>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ unsigned char smem_raw[];
+  griddep_wait();
+  griddep_launch_next();
   const uint32_t base = smem_u32(smem_raw);
   unsigned char *sbase = smem_raw;
   if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
@@ -677,7 +680,9 @@ cudaError_t launch_bwd_tc(const Problem &p, const BwdMaps &m, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t grid = p.bwd_slots < num_sms() ? p.bwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_bwd_tc<D, BF16, kCausal, kDQ><<<unsigned(grid), kBThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout, m.dq_acc);
+  e = launch_dep(k_bwd_tc<D, BF16, kCausal, kDQ>, dim3(unsigned(grid)), dim3(kBThreads), size_t(smem), s,
+                 p, m.q, m.k, m.v, m.dout, m.dq_acc);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@
 #include "bsa_internal.h"
 #include "fwd_walk.cuh"
 #include "f32x2.cuh"
+#include "launch.cuh"
 #include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -99,6 +100,8 @@ __global__ void __launch_bounds__(kDThreads, 1)
   using L = DLayout<D>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;
   extern __shared__ unsigned char smem_raw[];
+  griddep_wait();
+  griddep_launch_next();
   const uint32_t base = smem_u32(smem_raw);
   unsigned char *sbase = smem_raw;
   if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
@@ -424,7 +427,9 @@ cudaError_t launch_dq(const Problem &p, const DqMaps &m, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t grid = p.fwd_slots < num_sms() ? p.fwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_dq_tc<D, BF16, kCausal><<<unsigned(grid), kDThreads, smem, s>>>(p, m.q, m.k, m.v, m.dout);
+  e = launch_dep(k_dq_tc<D, BF16, kCausal>, dim3(unsigned(grid)), dim3(kDThreads), size_t(smem), s,
+                 p, m.q, m.k, m.v, m.dout);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

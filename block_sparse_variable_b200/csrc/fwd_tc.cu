@@ -41,6 +41,7 @@
 #include "bsa_internal.h"
 #include "fp8.cuh"
 #include "fwd_walk.cuh"
+#include "launch.cuh"
 #include "pack16.cuh"
 #include "sm100.cuh"
 #include "tc_common.h"
@@ -119,6 +120,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using L = Layout<D, kFp8>;
   using T = typename std::conditional<BF16, __nv_bfloat16, __half>::type;  // out (and 16-bit inputs)
   extern __shared__ unsigned char smem_raw[];
+  griddep_wait();
+  griddep_launch_next();
   const uint32_t base = smem_u32(smem_raw);
   unsigned char *sbase = smem_raw;
   if (base & 1023u) {  // 128-byte swizzled tiles need a 1024-byte aligned base
@@ -555,7 +558,9 @@ cudaError_t launch_tc2(const Problem &p, const FwdMaps &m, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t grid = p.fwd_slots < num_sms() ? p.fwd_slots : num_sms();
   if (grid <= 0) return cudaSuccess;
-  k_fwd_tc<D, BF16, kCausal, kFp8, kPack><<<unsigned(grid), kTcThreads, smem, s>>>(p, m.q, m.k, m.v);
+  e = launch_dep(k_fwd_tc<D, BF16, kCausal, kFp8, kPack>, dim3(unsigned(grid)), dim3(kTcThreads), size_t(smem), s,
+                 p, m.q, m.k, m.v);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

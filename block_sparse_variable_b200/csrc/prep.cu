@@ -15,6 +15,7 @@
 #include <cmath>
 
 #include "bsa_internal.h"
+#include "launch.cuh"
 
 namespace bsa {
 namespace {
@@ -22,6 +23,8 @@ namespace {
 __device__ __forceinline__ int64_t cdiv64(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 __global__ void k_geometry(Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   __shared__ uint32_t sflags;
   __shared__ int64_t s_sum_nq;
   uint32_t *st = p.status;
@@ -157,6 +160,8 @@ __device__ __forceinline__ uint64_t make_key(int32_t cost, int64_t id) {
 
 // one thread per (index head, global q-block row)
 __global__ void k_compact(Problem p, int fwd_keys) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t r = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (r >= int64_t(p.Hidx) * p.Rg) return;
   const int hi = int(r / p.Rg);
@@ -227,6 +232,8 @@ __device__ __forceinline__ bool row_has(const uint16_t *row, int n, int j) {
 // mode 0 counts the blocks and their 128-row query slices, mode 1 writes the
 // ascending list (ballots give each hit its place)
 __global__ void k_inverse(Problem p, int mode) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t idx = (int64_t(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (idx >= int64_t(p.Hidx) * p.tk_max) return;
@@ -271,6 +278,8 @@ __global__ void k_inverse(Problem p, int mode) {
 // single CTA exclusive scan of inv_cnt[0 .. Hidx*TK) into inv_off; also the
 // total of inv_sub (the backward work lists' grouping threshold)
 __global__ void k_scan_offsets(Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   __shared__ int32_t warp_sums[32];
   __shared__ int32_t carry;
   __shared__ unsigned long long sub_total;
@@ -336,6 +345,8 @@ __device__ __forceinline__ uint64_t bwd_key(int32_t cost, int h2, int64_t id, in
 
 // one thread per backward slot (h2, gk, kv slice)
 __global__ void k_bwd_keys(Problem p) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= p.bwd_slots) return;
   const int TK = int(p.status[kStTK]);
@@ -386,6 +397,8 @@ __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *
                                                                 uint64_t *sorted, int64_t slots,
                                                                 int n) {
   __shared__ uint64_t s[kSortChunk];
+  griddep_wait();
+  griddep_launch_next();
   const int t = threadIdx.x;
   const int64_t base = int64_t(blockIdx.x) * n;
   uint64_t v[4];
@@ -453,6 +466,8 @@ __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *
 // final position of every real key = its place in its chunk + the keys
 // below it in every other chunk (keys are unique: the id is in the low word)
 __global__ void k_rank(const uint64_t *sorted, int64_t nchunks, int n, int32_t *items) {
+  griddep_wait();
+  griddep_launch_next();
   const int64_t idx = int64_t(blockIdx.x) * blockDim.x + threadIdx.x;
   if (idx >= nchunks * n) return;
   const uint64_t key = sorted[idx];
@@ -476,14 +491,16 @@ __global__ void k_rank(const uint64_t *sorted, int64_t nchunks, int n, int32_t *
 }  // namespace
 
 cudaError_t launch_prep_geometry(const Problem &p, cudaStream_t s) {
-  k_geometry<<<1, 1024, 0, s>>>(p);
+  cudaError_t e = launch_dep(k_geometry, dim3(1), dim3(1024), 0, s, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep_compact(const Problem &p, bool fwd_keys, cudaStream_t s) {
   const int64_t n = int64_t(p.Hidx) * p.Rg;
   if (n > 0) {
-    k_compact<<<unsigned((n + 255) / 256), 256, 0, s>>>(p, fwd_keys ? 1 : 0);
+    cudaError_t e = launch_dep(k_compact, dim3(unsigned((n + 255) / 256)), dim3(256), 0, s, p, fwd_keys ? 1 : 0);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }
@@ -497,18 +514,25 @@ cudaError_t launch_sort_items(const Problem &p, int64_t slots_pad, int32_t *item
   int n = 128;
   while (n < slots && n < kSortChunk) n <<= 1;
   const int64_t nchunks = (slots + n - 1) / n;
-  k_sort_chunks<<<unsigned(nchunks), n / 4, 0, s>>>(p.keys, p.sorted, slots, n);
-  k_rank<<<unsigned((nchunks * n + 255) / 256), 256, 0, s>>>(p.sorted, nchunks, n, items);
+  cudaError_t e = launch_dep(k_sort_chunks, dim3(unsigned(nchunks)), dim3(unsigned(n / 4)), 0, s,
+                             (const uint64_t *)p.keys, p.sorted, slots, n);
+  if (e != cudaSuccess) return e;
+  e = launch_dep(k_rank, dim3(unsigned((nchunks * n + 255) / 256)), dim3(256), 0, s,
+                 (const uint64_t *)p.sorted, nchunks, n, items);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 cudaError_t launch_prep_inverse(const Problem &p, cudaStream_t s) {
   const int64_t n = int64_t(p.Hidx) * p.tk_max;  // lists, one warp each
   const unsigned grid = unsigned((n * 32 + 255) / 256);
-  if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 0);
-  k_scan_offsets<<<1, 1024, 0, s>>>(p);
-  if (n > 0) k_inverse<<<grid, 256, 0, s>>>(p, 1);
-  if (p.bwd_slots > 0) k_bwd_keys<<<unsigned((p.bwd_slots + 255) / 256), 256, 0, s>>>(p);
+  cudaError_t e = cudaSuccess;
+  if (n > 0 && (e = launch_dep(k_inverse, dim3(grid), dim3(256), 0, s, p, 0)) != cudaSuccess) return e;
+  if ((e = launch_dep(k_scan_offsets, dim3(1), dim3(1024), 0, s, p)) != cudaSuccess) return e;
+  if (n > 0 && (e = launch_dep(k_inverse, dim3(grid), dim3(256), 0, s, p, 1)) != cudaSuccess) return e;
+  if (p.bwd_slots > 0 &&
+      (e = launch_dep(k_bwd_keys, dim3(unsigned((p.bwd_slots + 255) / 256)), dim3(256), 0, s, p)) != cudaSuccess)
+    return e;
   return cudaGetLastError();
 }
 

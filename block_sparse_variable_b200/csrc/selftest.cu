@@ -4,6 +4,7 @@
 
 #include "bsa_internal.h"
 #include "exp2_poly.cuh"
+#include "f32x2.cuh"
 #include "fp8.cuh"
 #include "pack16.cuh"
 #include "tc_device.cuh"
@@ -46,6 +47,26 @@ __global__ void k_e4m3_pack(const float *x, uint32_t *y, int64_t nwords) {
     y[i] = pack_e4m3x4(x[4 * i], x[4 * i + 1], x[4 * i + 2], x[4 * i + 3]);
 }
 
+// the paired fp32 operations the backward's softmax uses, beside their scalar
+// forms: out[0..n) fma, [n..2n) add, [2n..3n) mul; pair = f32x2, scalar =
+// one rounding per element
+__global__ void k_f32x2_pair(const float *a, const float *b, const float *c, float *pair,
+                             float *scalar, int64_t n) {
+  for (int64_t i = blockIdx.x * int64_t(blockDim.x) + threadIdx.x; 2 * i < n;
+       i += int64_t(gridDim.x) * blockDim.x) {
+    const int64_t e = 2 * i;
+    const float2 A = make_float2(a[e], a[e + 1]), B = make_float2(b[e], b[e + 1]);
+    const float2 C = make_float2(c[e], c[e + 1]);
+    const float2 f = fma2(A, B, C), s = add2(A, B), m = mul2(A, B);
+    pair[e] = f.x, pair[e + 1] = f.y;
+    pair[n + e] = s.x, pair[n + e + 1] = s.y;
+    pair[2 * n + e] = m.x, pair[2 * n + e + 1] = m.y;
+    scalar[e] = __fmaf_rn(A.x, B.x, C.x), scalar[e + 1] = __fmaf_rn(A.y, B.y, C.y);
+    scalar[n + e] = __fadd_rn(A.x, B.x), scalar[n + e + 1] = __fadd_rn(A.y, B.y);
+    scalar[2 * n + e] = __fmul_rn(A.x, B.x), scalar[2 * n + e + 1] = __fmul_rn(A.y, B.y);
+  }
+}
+
 }  // namespace
 }  // namespace bsa
 
@@ -73,5 +94,17 @@ extern "C" bsa_status bsa_selftest_e4m3(const float *x, uint32_t *packed, int64_
   const int64_t w = n / 4;
   const int64_t blocks = (w + 255) / 256 < 1024 ? (w + 255) / 256 : 1024;
   bsa::k_e4m3_pack<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(x, packed, w);
+  return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
+}
+
+extern "C" bsa_status bsa_selftest_f32x2(const float *a, const float *b, const float *c,
+                                         float *pair, float *scalar, int64_t n, void *stream) {
+  if (n < 0 || n % 2 != 0) return BSA_ERR_PARAM_INVALID;
+  if (n == 0) return BSA_OK;
+  if (!a || !b || !c || !pair || !scalar) return BSA_ERR_NULLPTR;
+  const int64_t w = n / 2;
+  const int64_t blocks = (w + 255) / 256 < 1024 ? (w + 255) / 256 : 1024;
+  bsa::k_f32x2_pair<<<unsigned(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(a, b, c, pair,
+                                                                                     scalar, n);
   return cudaGetLastError() == cudaSuccess ? BSA_OK : BSA_ERR_CUDA;
 }

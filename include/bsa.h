@@ -344,6 +344,18 @@ bsa_status bsa_selftest_exp2(const float *x, float *y_poly, float *y_mufu, int64
  * uses for P.  n % 4 == 0; device pointers; asynchronous on `stream`. */
 bsa_status bsa_selftest_e4m3(const float *x, uint32_t *packed, int64_t n, void *stream);
 
+/* Diagnostic (the pages have no counterpart).  For n (even) float triples
+ * a[i], b[i], c[i] (device memory) writes, with the paired fp32 instructions
+ * of sm_100 (fma/add/mul .rn.f32x2, two elements per instruction) that the
+ * backward kernels' softmax uses, pair[i] = fma(a,b,c), pair[n+i] = a+b,
+ * pair[2n+i] = a*b, and the same three results from the scalar round-to-
+ * nearest operations into scalar[0..3n): the two must agree bit for bit.
+ * Caller-owned device buffers (pair and scalar 3n floats each); asynchronous
+ * on `stream`; BSA_ERR_PARAM_INVALID for n < 0 or odd, BSA_ERR_NULLPTR for a
+ * NULL buffer with n > 0, BSA_ERR_CUDA if the launch fails. */
+bsa_status bsa_selftest_f32x2(const float *a, const float *b, const float *c, float *pair,
+                              float *scalar, int64_t n, void *stream);
+
 /* Diagnostic (the pages have no counterpart).  Launches one warp that waits
  * on a device barrier nothing ever completes, through the bounded wait every
  * kernel of this library uses: after its time limit (about 2 s) the wait
