@@ -27,7 +27,8 @@ __device__ __forceinline__ int64_t qstore_off(const Problem &p, int64_t sb, int6
 
 // eight lanes per (query row, head): each reads 16 bytes of dOut and out per
 // pass (a warp covers four (row, head) pairs, 512 bytes of each tensor per
-// pass), then the eight partial dot products are summed by shuffles
+// pass), then the eight partial dot products are summed by shuffles; the
+// same lanes zero the pair's row of the fp32 dQ accumulator
 template <typename T>
 __global__ void k_bwd_pre(const Problem p) {
   griddep_wait();
@@ -53,6 +54,12 @@ __global__ void k_bwd_pre(const Problem p) {
         const float2 y = Pack2<T>::unpack(cv[e]);
         acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
       }
+    }
+    // the pair's fp32 dQ accumulator row starts at zero (the same eight
+    // lanes, 16 bytes each per pass)
+    if (p.dq_acc) {
+      uint4 *acc_row = reinterpret_cast<uint4 *>(p.dq_acc + w * p.D);
+      for (int d = sub * 4; d < p.D; d += 32) acc_row[d / 4] = make_uint4(0, 0, 0, 0);
     }
   }
 #pragma unroll
@@ -115,11 +122,9 @@ __global__ void k_kv_zero_tail(const Problem p) {
 
 }  // namespace
 
+// (the dQ accumulator, absent in the deterministic backward, is zeroed by
+// the same kernel)
 cudaError_t launch_bwd_pre(const Problem &p, cudaStream_t s) {
-  if (p.dq_acc) {  // absent in the deterministic backward (dq written directly)
-    cudaError_t e = cudaMemsetAsync(p.dq_acc, 0, size_t(p.rows_q) * p.N1 * p.D * sizeof(float), s);
-    if (e != cudaSuccess) return e;
-  }
   const int64_t pairs = p.rows_q * p.N1;  // eight lanes each
   const unsigned grid = unsigned((pairs * 8 + 255) / 256);
   cudaError_t e = p.dtype == BSA_BF16 ? launch_dep(k_bwd_pre<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, p)
