@@ -393,9 +393,11 @@ __device__ __forceinline__ uint64_t shfl_xor64(uint64_t x, int m) {
 // registers.  Stages whose partner distance j is 1 or 2 stay in the thread,
 // 4 <= j <= 64 cross lanes of one warp (shuffles), j >= 128 go through shared
 // memory, where consecutive such stages run in place.
+// A single chunk is the whole list: its sorted keys go straight to the item
+// list (`items`, else null), each real key's place being its rank.
 __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *keys,
                                                                 uint64_t *sorted, int64_t slots,
-                                                                int n) {
+                                                                int n, int32_t *items) {
   __shared__ uint64_t s[kSortChunk];
   griddep_wait();
   griddep_launch_next();
@@ -418,7 +420,10 @@ __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *
     if ((t & 31) == 31 && t + 1 < int(blockDim.x)) in_order = in_order && v[3] <= s[(t >> 5) + 1];
     if (__syncthreads_and(in_order)) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) sorted[base + 4 * t + r] = v[r];
+      for (int r = 0; r < 4; ++r) {
+        if (!items) sorted[base + 4 * t + r] = v[r];
+        else if (v[r] != kAbsentKey) items[4 * t + r] = int32_t(uint32_t(v[r] & 0xFFFFFFFFu));
+      }
       return;
     }
   }
@@ -460,7 +465,10 @@ __global__ void __launch_bounds__(kSortChunk / 4) k_sort_chunks(const uint64_t *
     cmp_swap(v[2], v[3], k == 2 ? false : up);
   }
 #pragma unroll
-  for (int r = 0; r < 4; ++r) sorted[base + 4 * t + r] = v[r];
+  for (int r = 0; r < 4; ++r) {
+    if (!items) sorted[base + 4 * t + r] = v[r];
+    else if (v[r] != kAbsentKey) items[4 * t + r] = int32_t(uint32_t(v[r] & 0xFFFFFFFFu));
+  }
 }
 
 // final position of every real key = its place in its chunk + the keys
@@ -515,11 +523,14 @@ cudaError_t launch_sort_items(const Problem &p, int64_t slots_pad, int32_t *item
   while (n < slots && n < kSortChunk) n <<= 1;
   const int64_t nchunks = (slots + n - 1) / n;
   cudaError_t e = launch_dep(k_sort_chunks, dim3(unsigned(nchunks)), dim3(unsigned(n / 4)), 0, s,
-                             (const uint64_t *)p.keys, p.sorted, slots, n);
+                             (const uint64_t *)p.keys, p.sorted, slots, n,
+                             nchunks == 1 ? items : (int32_t *)nullptr);
   if (e != cudaSuccess) return e;
-  e = launch_dep(k_rank, dim3(unsigned((nchunks * n + 255) / 256)), dim3(256), 0, s,
-                 (const uint64_t *)p.sorted, nchunks, n, items);
-  if (e != cudaSuccess) return e;
+  if (nchunks > 1) {
+    e = launch_dep(k_rank, dim3(unsigned((nchunks * n + 255) / 256)), dim3(256), 0, s,
+                   (const uint64_t *)p.sorted, nchunks, n, items);
+    if (e != cudaSuccess) return e;
+  }
   return cudaGetLastError();
 }
 
