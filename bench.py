@@ -42,11 +42,25 @@ DESCR = {
     4: "C4: BNSD B=1 N1=N2=24 S=32768 D=128 bf16, block (128,128), sink+diag+14 random of 256",
     5: "C5: TND q B=8 lens U[512,4096] + paged KV [P,128,8,128] fp16, N1=32 N2=8, top-8 blocks",
 }
-# kernels this library launches per step (forward 5, backward 12; the
-# deterministic backward 14: the forward list's sort and the dQ pass added,
-# the dQ conversion dropped)
-LAUNCHES_PER_STEP = 17
-LAUNCHES_PER_STEP_DET = 19
+# kernels this library launches per call: forward geometry, compaction, sort
+# (+ the rank merge when the list spans more than one 4096-key chunk), main;
+# backward geometry, compaction, inverse count, scan, inverse fill, keys,
+# sort (+ rank), preprocessing, main, dQ conversion, kv tail; the
+# deterministic backward adds the forward list's sort (+ rank) and the dQ
+# pass and drops the dQ conversion
+SORT_CHUNK = 4096
+
+
+def _sort_launches(slots: int) -> int:
+    return 0 if slots == 0 else (1 if slots <= SORT_CHUNK else 2)
+
+
+def launches_per_step(fwd_slots: int, bwd_slots: int, deterministic: bool) -> int:
+    fwd = 3 + _sort_launches(fwd_slots)
+    bwd = 10 + _sort_launches(bwd_slots)
+    if deterministic:
+        bwd += _sort_launches(fwd_slots)
+    return fwd + bwd
 
 
 def _peaks():
@@ -382,6 +396,9 @@ def run_ours(args):
     wsb = torch.empty(bsa.bsa_bwd_get_workspace(q, k, v, out, dout, lse, index, P, dq=dq, dk=dk,
                                                 dv=dv, **opt), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
+    # the work lists' slot counts (their regions hold one int32 per slot)
+    fwd_slots = bsa.bsa_fwd_workspace_layout(q, k, v, index, P, out=out, lse=lse, **opt).fwd_items.bytes // 4
+    bwd_slots = bsa.bsa_bwd_workspace_layout(q, k, v, out, dout, lse, index, P, **opt).bwd_items.bytes // 4
 
     def step():
         bsa.bsa_fwd(q, k, v, index, P, out=out, lse=lse, workspace=wsf, stream=stream, **opt)
@@ -516,7 +533,7 @@ def run_ours(args):
             "e2e": {"value": round(job_tflops(world, step_flops, e2e_ms), 3), "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": round(e2e_ms, 3)},
-            "gpu_launches": (LAUNCHES_PER_STEP_DET if args.deterministic else LAUNCHES_PER_STEP) * args.steps,
+            "gpu_launches": launches_per_step(fwd_slots, bwd_slots, args.deterministic) * args.steps,
             "status_flags": flags,
             "clocks": clk.summary(),
         }
@@ -551,6 +568,7 @@ def run_fp8(args):
     lse = torch.empty(q.shape[:3], dtype=torch.float32, device=dev)
     wsf = torch.empty(bsa.bsa_fwd_get_workspace(q, k, v, index, P, out=out, lse=lse),
                       dtype=torch.uint8, device=dev)
+    fwd_slots = bsa.bsa_fwd_workspace_layout(q, k, v, index, P, out=out, lse=lse).fwd_items.bytes // 4
     stream = torch.cuda.current_stream()
 
     def step():
@@ -620,7 +638,8 @@ def run_fp8(args):
                      "peak_source": f"{which} bf16 burst x 2 (nominal fp8/bf16 ratio)", "traffic": None},
         "e2e": {"value": round(flops / (e2e_ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3)},
-        "gpu_launches": 5 * args.steps, "status_flags": flags, "clocks": clk.summary(),
+        "gpu_launches": (3 + _sort_launches(fwd_slots)) * args.steps, "status_flags": flags,
+        "clocks": clk.summary(),
     }
     if not args.no_cpu_baseline:
         import oracle

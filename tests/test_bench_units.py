@@ -72,3 +72,12 @@ def test_oracle_sample_takes_whole_heads_past_one_head():
     one = bench._oracle_subproblem(3, 1024)
     assert one.N1 == 1 and bench._pairs(one) == 1024 * 8192
     assert torch.equal(one.q[0, 0], sub.q[0, 0, :1024])
+
+
+def test_launch_count_follows_the_sort_chunks():
+    """One sort launch for a list of up to 4096 slots, a sort and a rank
+    merge above; C3's lists have 4096 slots each, C4's 6144."""
+    assert bench.launches_per_step(4096, 4096, False) == 15
+    assert bench.launches_per_step(6144, 6144, False) == 17
+    assert bench.launches_per_step(4096, 4096, True) == 16
+    assert bench.launches_per_step(6144, 6144, True) == 19
