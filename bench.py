@@ -270,7 +270,7 @@ def _descr(cfg: int, causal: bool, deterministic: bool = False, shared_rows: boo
                if per_head_rows else ""))
 
 
-def cpu_baseline(cfg: int, target_s: float = 12.0, causal: bool = False, shared_rows: bool = False):
+def cpu_baseline(cfg: int, target_s: float = 16.0, causal: bool = False, shared_rows: bool = False):
     sub, pairs = _oracle_rate(cfg, target_s, causal, shared_rows)
     t = _oracle_step(sub)
     flops = 14 * sub.D * pairs
