@@ -335,56 +335,82 @@ __global__ void __launch_bounds__(kBThreads, 1)
         tma_load_5d(sV, &map_v, bar(kBarKV), 0, row, 0, v.h2, last);
       }
       ++kv_it;
-      for (BStep c = b_settle(p, v, BStep{0, 0, 0}, TK); c.hh < p.g && ok; c = b_next(p, v, c, TK)) {
-        const int slot = int(sk & 1u);
-        const int h1 = v.h2 * p.g + c.hh;
-        const int t0 = b_t0(p, v, c, TK);
-        // lse (log2 units) and Dsum of the step's 128 query rows, fetched
-        // before waiting for the slot; rows past qlen get lse = +inf (so
-        // P = 0) and Dsum = 0.  Both are staged negated, as the addends of
-        // the softmax warps' paired fp32 operations.
-        float l2r[4], dsr[4];
+      // A step's inputs: its q head and first query row (the walk of the
+      // inverted index) and the raw lse / Dsum of its 128 query rows (rows
+      // past qlen: lse -inf, Dsum 0).  They are fetched one step ahead: with
+      // the dQ product, while the TMA unit reads the previous dQ out of the
+      // slot, so that the walk's dependent loads are not on the slot's path.
+      auto fetch = [&](const BStep &c, int &h1, int &t0, float (&l2r)[4], float (&dsr)[4]) {
+        h1 = v.h2 * p.g + c.hh;
+        t0 = b_t0(p, v, c, TK);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int t = t0 + lane + 32 * i;
-          l2r[i] = INFINITY;
+          l2r[i] = -INFINITY;
           dsr[i] = 0.f;
           if (t < v.bi.qlen) {
-            const float l2 = p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, h1, t)] * kLog2e;
-            l2r[i] = l2 > -INFINITY ? l2 : INFINITY;  // a row with no selected key
+            l2r[i] = p.lse[q_row(p.l_sb, p.l_sh, p.l_st, v.bi, v.b, h1, t)];
             const int64_t srow = p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq + t : v.bi.q_tok0 + t;
             dsr[i] = p.dsum[srow * p.N1 + h1];
           }
         }
+      };
+      BStep c = b_settle(p, v, BStep{0, 0, 0}, TK);
+      int h1 = 0, t0 = 0;
+      float l2r[4], dsr[4];
+      if (c.hh < p.g) fetch(c, h1, t0, l2r, dsr);
+      while (c.hh < p.g && ok) {
+        const int slot = int(sk & 1u);
         // the step that held the slot before: its dQ is staged over the
         // slot's tiles; hand it to the TMA unit in two commit groups (Q tile,
         // dOut tile) so that each tile is refilled as soon as it is read out
         const bool refill = sk >= 2;
         if (refill && !(ok = wait_warp_lazy(bar(kBarDQOut + slot), ((sk - 2) >> 1) & 1u, abort, p.status))) break;
+        // lse in log2 units, +inf for rows past qlen or with no selected key
+        // (so P = 0), and Dsum; both staged negated, as the addends of the
+        // softmax warps' paired fp32 operations
         float *st = stat + slot * 256;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          st[lane + 32 * i] = -l2r[i];
+          const float l2 = l2r[i] * kLog2e;
+          st[lane + 32 * i] = -(l2 > -INFINITY ? l2 : INFINITY);
           st[128 + lane + 32 * i] = -dsr[i];
         }
         if constexpr (!kDQ)
           if (lane == 0) step_t0[slot] = t0;
         __syncwarp();
+        const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
+        const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
         if (lane == 0) {
           if (kDQ && refill) reduce_slot(slot);
           mbar_expect_tx(bar(kBarQD + slot), 2 * L::kTile);
           armed_qd[slot] = int((sk >> 1) & 1u);
-          const int tok = p.q_layout == BSA_LAYOUT_TND ? int(v.bi.q_tok0) + t0 : t0;
-          const int bb = p.q_layout == BSA_LAYOUT_TND ? 0 : v.b;
+        }
+        __syncwarp();
+        const bool ahead = kDQ && refill;  // fetch while the slot is read out
+        const BStep cn = b_next(p, v, c, TK);
+        int h1n = 0, t0n = 0;
+        float l2n[4] = {0.f, 0.f, 0.f, 0.f}, dsn[4] = {0.f, 0.f, 0.f, 0.f};
+        if (ahead && cn.hh < p.g) fetch(cn, h1n, t0n, l2n, dsn);
+        if (lane == 0) {
           if (kDQ && refill) bulk_wait_read<1>();
           tma_load_5d(sQ + slot * L::kTile, &map_q, bar(kBarQD + slot), 0, tok, 0, h1, bb);
           if (kDQ && refill) bulk_wait_read<0>();
           tma_load_5d(sDO + slot * L::kTile, &map_do, bar(kBarQD + slot), 0, tok, 0, h1, bb);
         }
         __syncwarp();
+        if (!ahead && cn.hh < p.g) fetch(cn, h1n, t0n, l2n, dsn);
         pend_h[slot] = h1;
         pend_row[slot] = int((p.q_layout == BSA_LAYOUT_BNSD ? int64_t(v.b) * p.Sq : v.bi.q_tok0) + t0);
         ++sk;
+        c = cn;
+        h1 = h1n;
+        t0 = t0n;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          l2r[i] = l2n[i];
+          dsr[i] = dsn[i];
+        }
       }
     }
     if (kDQ)
